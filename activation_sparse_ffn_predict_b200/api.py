@@ -1,0 +1,187 @@
+"""Tensor-level binding of the asffn C ABI (same names as include/asffn.h).
+
+torch supplies device memory and streams; every step of the path runs in
+libasffn.so's CUDA kernels.  These wrappers only check that tensors live where
+the C ABI expects them (device or host), build the descriptor structs and
+marshal pointers; a non-OK status raises ``AsfError``.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import _lib as L
+from ._lib import AsfError, check  # noqa: F401
+
+_DT = {torch.float16: L.ASF_F16, torch.float32: L.ASF_F32}
+_ACT = {"relu": L.ASF_ACT_RELU, "reglu": L.ASF_ACT_REGLU}
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> ctypes.c_void_p:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+class Predictor:
+    """Descriptor of the two-layer predictor: W1 [r,d], b1 [r], W2 [n,r], b2 [n]."""
+
+    def __init__(self, W1: torch.Tensor, b1: torch.Tensor, W2: torch.Tensor, b2: torch.Tensor):
+        if W1.dtype not in _DT or W2.dtype != W1.dtype:
+            raise ValueError("W1/W2 must both be float16 or float32")
+        r, d = W1.shape
+        n, r2 = W2.shape
+        if r2 != r or b1.shape != (r,) or b2.shape != (n,):
+            raise ValueError("predictor shapes do not agree")
+        self.tensors = (W1, b1, W2, b2)
+        self.d, self.r, self.n, self.dtype = d, r, n, W1.dtype
+        self.desc = L.asf_predictor(d, r, n, _DT[W1.dtype], _dev(W1, "W1"),
+                                    _dev(b1, "b1", torch.float32), _dev(W2, "W2"),
+                                    _dev(b2, "b2", torch.float32))
+
+
+class FFN:
+    """Descriptor of one FFN layer in storage order: Wg/Wu/WdT [n,d], bias [n]."""
+
+    def __init__(self, act: str, Wg: Optional[torch.Tensor], Wu: torch.Tensor, WdT: torch.Tensor,
+                 bias: torch.Tensor):
+        if act not in _ACT:
+            raise ValueError("act must be 'reglu' or 'relu'")
+        if Wu.dtype not in _DT or WdT.dtype != Wu.dtype:
+            raise ValueError("weights must be float16 or float32")
+        n, d = Wu.shape
+        if WdT.shape != (n, d) or bias.shape != (n,):
+            raise ValueError("FFN shapes do not agree")
+        if act == "reglu":
+            if Wg is None or Wg.shape != (n, d) or Wg.dtype != Wu.dtype:
+                raise ValueError("ReGLU needs a gate matrix shaped like W_up")
+            gp = _dev(Wg, "Wg")
+        else:
+            gp = ctypes.c_void_p(0)
+        self.tensors = (Wg, Wu, WdT, bias)
+        self.act, self.d, self.n, self.dtype = act, d, n, Wu.dtype
+        self.desc = L.asf_ffn(d, n, _DT[Wu.dtype], _ACT[act], gp, _dev(Wu, "Wu"), _dev(WdT, "WdT"),
+                              _dev(bias, "bias", torch.float32))
+
+
+def asf_version() -> int:
+    return int(L.load().asf_version())
+
+
+def asf_workspace_bytes(pred: Optional[Predictor], ffn: Optional[FFN], max_batch: int) -> int:
+    lib = L.load()
+    p = ctypes.byref(pred.desc) if pred is not None else None
+    f = ctypes.byref(ffn.desc) if ffn is not None else None
+    return int(lib.asf_workspace_bytes(p, f, int(max_batch)))
+
+
+class Workspace:
+    """Device scratch for one stream: sized by asf_workspace_bytes, zeroed once."""
+
+    def __init__(self, pred: Optional[Predictor], ffn: Optional[FFN], max_batch: int, device=None,
+                 stream=None):
+        nbytes = asf_workspace_bytes(pred, ffn, max_batch)
+        if nbytes == 0:
+            raise AsfError(L.ASF_ERR_INVALID_ARG, "asf_workspace_bytes")
+        dev = device if device is not None else (ffn or pred).tensors[-1].device
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.nbytes = nbytes
+        asf_workspace_init(self, stream)
+
+    @property
+    def ptr(self) -> ctypes.c_void_p:
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+
+def asf_workspace_init(ws: Workspace, stream=None) -> None:
+    check(L.load().asf_workspace_init(ws.ptr, ws.nbytes, _stream(stream)), "asf_workspace_init")
+
+
+def asf_predict(pred: Predictor, x: torch.Tensor, tau: float, idx: torch.Tensor, count: torch.Tensor,
+                ws: Workspace, stream=None) -> None:
+    """idx[:count] = ascending union of neurons with sigmoid(W2 ReLU(W1 x + b1) + b2) > tau."""
+    if x.dtype != pred.dtype or x.dim() != 2 or x.shape[1] != pred.d:
+        raise ValueError("x must be [B, d] in the predictor's dtype")
+    st = L.load().asf_predict(ctypes.byref(pred.desc), _dev(x, "x"), int(x.shape[0]), float(tau),
+                              _dev(idx, "idx", torch.int32), _dev(count, "count", torch.int32),
+                              ws.ptr, ws.nbytes, _stream(stream))
+    check(st, "asf_predict")
+
+
+def asf_sparse_ffn(ffn: FFN, x: torch.Tensor, idx: torch.Tensor, count: torch.Tensor, y: torch.Tensor,
+                   ws: Workspace, stream=None) -> None:
+    """y = sum over the first count entries k of idx of a_k(x) * WdT[k]."""
+    if x.dtype != ffn.dtype or x.dim() != 2 or x.shape[1] != ffn.d:
+        raise ValueError("x must be [B, d] in the FFN's dtype")
+    if y.shape != (x.shape[0], ffn.d):
+        raise ValueError("y must be [B, d]")
+    st = L.load().asf_sparse_ffn(ctypes.byref(ffn.desc), _dev(x, "x"), int(x.shape[0]),
+                                 _dev(idx, "idx", torch.int32), _dev(count, "count", torch.int32),
+                                 _dev(y, "y", torch.float32), ws.ptr, ws.nbytes, _stream(stream))
+    check(st, "asf_sparse_ffn")
+
+
+def asf_dense_ffn(ffn: FFN, x: torch.Tensor, y: torch.Tensor, ws: Workspace, stream=None) -> None:
+    if x.dtype != ffn.dtype or x.dim() != 2 or x.shape[1] != ffn.d or y.shape != (x.shape[0], ffn.d):
+        raise ValueError("x must be [B, d] in the FFN's dtype and y [B, d]")
+    st = L.load().asf_dense_ffn(ctypes.byref(ffn.desc), _dev(x, "x"), int(x.shape[0]),
+                                _dev(y, "y", torch.float32), ws.ptr, ws.nbytes, _stream(stream))
+    check(st, "asf_dense_ffn")
+
+
+def asf_activation_counts(ffn: FFN, x: torch.Tensor, counts: torch.Tensor, ws: Workspace,
+                          stream=None) -> None:
+    """counts[k] += #tokens of x whose ReLU input for neuron k is > 0."""
+    if x.dtype != ffn.dtype or x.dim() != 2 or x.shape[1] != ffn.d or counts.shape != (ffn.n,):
+        raise ValueError("x must be [T, d] in the FFN's dtype and counts [n]")
+    st = L.load().asf_activation_counts(ctypes.byref(ffn.desc), _dev(x, "x"), int(x.shape[0]),
+                                        _dev(counts, "counts", torch.int64), ws.ptr, ws.nbytes,
+                                        _stream(stream))
+    check(st, "asf_activation_counts")
+
+
+def asf_hot_permutation(counts) -> np.ndarray:
+    """Host: neuron ids by descending count, ties to the lower id."""
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.int64))
+    out = np.empty(c.shape[0], dtype=np.int32)
+    st = L.load().asf_hot_permutation(c.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), int(c.shape[0]),
+                                      out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+    check(st, "asf_hot_permutation")
+    return out
+
+
+def asf_permute_rows(src: torch.Tensor, dst: torch.Tensor, perm: torch.Tensor, stream=None) -> None:
+    """dst[i] = src[perm[i]] (row gather on the device)."""
+    if src.shape != dst.shape or src.dtype != dst.dtype or src.shape[0] != perm.shape[0]:
+        raise ValueError("src/dst must match and have one row per perm entry")
+    n_rows = int(src.shape[0])
+    row_bytes = src.numel() * src.element_size() // max(1, n_rows)
+    st = L.load().asf_permute_rows(_dev(src, "src"), _dev(dst, "dst"), n_rows, row_bytes,
+                                   _dev(perm, "perm", torch.int32), _stream(stream))
+    check(st, "asf_permute_rows")
+
+
+def asf_read_error(ws: Workspace, stream=None) -> int:
+    """Synchronise the stream, return and clear the device error status (0 = none)."""
+    out = ctypes.c_int32(0)
+    check(L.load().asf_read_error(ws.ptr, ctypes.byref(out), _stream(stream)), "asf_read_error")
+    return int(out.value)
+
+
+def asf_status_string(status: int) -> str:
+    return L.load().asf_status_string(int(status)).decode()

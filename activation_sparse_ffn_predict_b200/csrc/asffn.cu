@@ -1,0 +1,940 @@
+// libasffn: activation-sparse FFN decode path for B200 (sm_100a).
+//
+// Operations (see include/asffn.h for the ABI contract):
+//   predictor layer 1   h = ReLU(W1 x + b1)                 k_pred_l1
+//   predictor layer 2   z = W2 h + b2, z > logit(tau),       k_pred_l2
+//                       union over tokens, ascending compaction by the last CTA
+//   gate/up gather      a_k = ReLU(Wg[k].x + b_k) * Wu[k].x  k_ffn_gu
+//                       (or ReLU(Wu[k].x + b_k)) for k in idx
+//   down accumulate     y = sum_j a_j WdT[idx_j]             k_ffn_down
+//   profiler            counts[k] += #(ReLU input > 0)       k_act_counts
+//   row gather          dst[i] = src[perm[i]]                k_permute_rows
+//
+// Method: "PowerInfer Guide: Exploiting Activation Sparsity for LLM AI" (FFN
+// equation in "The Hidden Inefficiency"; predictor equation in section 3
+// "Adaptive Online Neuron Predictors"; section 4 "Neuron-Aware Sparse GPU
+// Operators"; Step 1 profiler) and the 2-layer MLP predictor of the
+// "PowerInfer_x64" page.  The kernels are this library's own B200 design:
+// every weight byte is streamed once with 16-byte non-allocating loads, the
+// activation vector lives in shared memory, accumulation is fp32, and every
+// cross-CTA reduction is deterministic (fixed-order sums by the last CTA to
+// finish, found with an atomic ticket; no spin-waits, no float atomics).
+// Consecutive kernels overlap through programmatic dependent launch: each
+// kernel may prefetch its weights into L2 before waiting for its inputs.
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "asffn.h"
+#include "common.cuh"
+
+using namespace asf;
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / kWarp;
+constexpr int kMaxSplits = 64;        // max CTAs summing into one column tile
+constexpr int kTargetCtas = 296;      // 2 CTAs on each of the 148 SMs
+constexpr size_t kSmemBudget = 96 * 1024;
+
+// ======================================================================== //
+// shared building blocks                                                   //
+// ======================================================================== //
+
+// Dot products of one weight row with NB activation vectors held in shared
+// memory in the weight's own 16-byte chunk layout.  Lane l handles chunks
+// l, l+32, ...; U chunks are in flight per lane.  Returns lane partial sums.
+template <typename T, int NB, int U>
+__device__ __forceinline__ void row_dot(const T *__restrict__ w, const T *xs, int xs_stride,
+                                        int nvec, int lane, float (&acc)[NB]) {
+  constexpr int V = Vec<T>::N;
+  int c = lane;
+  for (; c + (U - 1) * kWarp < nvec; c += U * kWarp) {
+    uint4 wv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) wv[u] = ld_stream(w + (size_t)(c + u * kWarp) * V);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const uint4 xv =
+            *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)(c + u * kWarp) * V);
+        acc[b] = Vec<T>::dot(wv[u], xv, acc[b]);
+      }
+    }
+  }
+  for (; c < nvec; c += kWarp) {
+    const uint4 wv = ld_stream(w + (size_t)c * V);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)c * V);
+      acc[b] = Vec<T>::dot(wv, xv, acc[b]);
+    }
+  }
+}
+
+// Same for two rows sharing the activation loads (gate and up of one neuron).
+template <typename T, int NB, int U>
+__device__ __forceinline__ void row_dot2(const T *__restrict__ w0, const T *__restrict__ w1,
+                                         const T *xs, int xs_stride, int nvec, int lane,
+                                         float (&acc0)[NB], float (&acc1)[NB]) {
+  constexpr int V = Vec<T>::N;
+  int c = lane;
+  for (; c + (U - 1) * kWarp < nvec; c += U * kWarp) {
+    uint4 wa[U], wb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      wa[u] = ld_stream(w0 + (size_t)(c + u * kWarp) * V);
+      wb[u] = ld_stream(w1 + (size_t)(c + u * kWarp) * V);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const uint4 xv =
+            *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)(c + u * kWarp) * V);
+        acc0[b] = Vec<T>::dot(wa[u], xv, acc0[b]);
+        acc1[b] = Vec<T>::dot(wb[u], xv, acc1[b]);
+      }
+    }
+  }
+  for (; c < nvec; c += kWarp) {
+    const uint4 wa = ld_stream(w0 + (size_t)c * V);
+    const uint4 wb = ld_stream(w1 + (size_t)c * V);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)c * V);
+      acc0[b] = Vec<T>::dot(wa, xv, acc0[b]);
+      acc1[b] = Vec<T>::dot(wb, xv, acc1[b]);
+    }
+  }
+}
+
+// Copy tokens [g0, g0+nb) of x ([B][d], dtype T) into shared memory [NB][d],
+// zero-filling the unused token slots.  x may come from the previous kernel,
+// so it is read through L2.
+template <typename T, int NB>
+__device__ __forceinline__ void stage_tokens(T *xs, const T *__restrict__ x, int d, int g0, int nb) {
+  constexpr int V = Vec<T>::N;
+  const int nvec = d / V;
+  for (int i = threadIdx.x; i < NB * nvec; i += blockDim.x) {
+    const int b = i / nvec;
+    const int c = i - b * nvec;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (b < nb) v = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)(g0 + b) * d + (size_t)c * V));
+    *reinterpret_cast<uint4 *>(xs + (size_t)b * d + (size_t)c * V) = v;
+  }
+}
+
+// Spread an L2 prefetch of [p, p + bytes) over the CTA's threads in 16 KB
+// pieces (bytes is a multiple of 16, p 16-byte aligned).
+__device__ __forceinline__ void prefetch_range(const void *p, size_t bytes) {
+  constexpr size_t kPiece = 16384;
+  const unsigned char *c = static_cast<const unsigned char *>(p);
+  for (size_t o = (size_t)threadIdx.x * kPiece; o < bytes; o += (size_t)blockDim.x * kPiece)
+    prefetch_l2(c + o, (uint32_t)min(kPiece, bytes - o));
+}
+
+// ======================================================================== //
+// predictor                                                                //
+// ======================================================================== //
+
+// Layer 1: h[b][i] = max(W1[i] . x[b] + b1[i], 0).  CTA c owns rows
+// [c*rpc, (c+1)*rpc); warps take rows round-robin.  Also clears the union mask
+// that layer 2 fills.
+template <typename T, int NB, int U>
+__global__ void __launch_bounds__(kThreads)
+    k_pred_l1(const T *__restrict__ W1, const float *__restrict__ b1, const T *__restrict__ x, int d,
+              int r, int B, int rpc, float *__restrict__ h, uint32_t *__restrict__ mask_words,
+              int n_words, int prefetch) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  T *xs = reinterpret_cast<T *>(smem_raw);
+  constexpr int V = Vec<T>::N;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row0 = blockIdx.x * rpc;
+  const int row1 = min(r, row0 + rpc);
+  if (prefetch && row0 < row1) prefetch_range(W1 + (size_t)row0 * d, (size_t)(row1 - row0) * d * sizeof(T));
+  pdl_wait();
+  pdl_trigger();
+  for (int w = blockIdx.x * kThreads + threadIdx.x; w < n_words; w += gridDim.x * kThreads)
+    mask_words[w] = 0u;
+  const int nvec = d / V;
+  for (int g0 = 0; g0 < B; g0 += NB) {
+    const int nb = min(NB, B - g0);
+    __syncthreads();
+    stage_tokens<T, NB>(xs, x, d, g0, nb);
+    __syncthreads();
+    for (int row = row0 + warp; row < row1; row += kWarps) {
+      float acc[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+      row_dot<T, NB, U>(W1 + (size_t)row * d, xs, d, nvec, lane, acc);
+      const float bias = __ldg(b1 + row);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float s = warp_sum(acc[b]);
+        if (lane == b && b < nb) h[(size_t)(g0 + b) * r + row] = fmaxf(s + bias, 0.f);
+      }
+    }
+  }
+}
+
+// Stage h[g0..g0+nb) ([B][r] fp32) for dot products with rows of T.  For fp16
+// rows (8 elements per 16-byte chunk) the 8 floats of chunk c are split into
+// two planes of 4 so that a warp's shared-memory reads are conflict-free.
+template <typename T, int NB>
+__device__ __forceinline__ void stage_hidden(float *hs, const float *__restrict__ h, int r, int g0, int nb) {
+  for (int i = threadIdx.x; i < NB * r; i += blockDim.x) {
+    const int b = i / r;
+    const int e = i - b * r;
+    const float v = (b < nb) ? __ldcg(h + (size_t)(g0 + b) * r + e) : 0.f;
+    int pos = e;
+    if (sizeof(T) == 2) {
+      const int c = e >> 3, q = e & 7;
+      pos = (q < 4) ? (c * 4 + q) : (r / 2 + c * 4 + (q - 4));
+    }
+    hs[(size_t)b * r + pos] = v;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float dot_hidden(uint4 w, const float *hsb, int r, int c) {
+  if constexpr (sizeof(T) == 2) {
+    return Vec<__half>::dotf2(w, hsb + c * 4, hsb + r / 2 + c * 4, 0.f);
+  } else {
+    return Vec<float>::dotf(w, hsb + c * 4, 0.f);
+  }
+}
+
+// Layer 2 + threshold + union + compaction.  CTA c owns rows [c*rpc, ...);
+// each warp computes R rows at a time.  Bits of rows predicted active for any
+// token are OR-ed into the global union mask; the last CTA to finish (atomic
+// ticket, no waiting) turns the mask into the ascending index list.
+template <typename T, int NB, int R>
+__global__ void __launch_bounds__(kThreads)
+    k_pred_l2(const T *__restrict__ W2, const float *__restrict__ b2, const float *__restrict__ h,
+              int r, int n, int B, float thr, int rpc, uint32_t *__restrict__ mask_words, int n_words,
+              int32_t *__restrict__ idx, int32_t *__restrict__ count, Header *__restrict__ hdr,
+              int prefetch) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float *hs = reinterpret_cast<float *>(smem_raw);
+  uint32_t *smask = reinterpret_cast<uint32_t *>(hs + (size_t)NB * r);
+  __shared__ int s_last;
+  __shared__ int s_wsum[kWarps];
+  constexpr int V = Vec<T>::N;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row0 = blockIdx.x * rpc;
+  const int row1 = min(n, row0 + rpc);
+  if (prefetch && row0 < row1) prefetch_range(W2 + (size_t)row0 * r, (size_t)(row1 - row0) * r * sizeof(T));
+  const int wfirst = row0 >> 5;
+  const int nwl = (row0 < row1) ? (((row1 - 1) >> 5) - wfirst + 1) : 0;
+  for (int i = threadIdx.x; i < nwl; i += kThreads) smask[i] = 0u;
+  pdl_wait();
+  pdl_trigger();
+  const int nvec = r / V;
+  for (int g0 = 0; g0 < B; g0 += NB) {
+    const int nb = min(NB, B - g0);
+    __syncthreads();
+    stage_hidden<T, NB>(hs, h, r, g0, nb);
+    __syncthreads();
+    for (int rb = row0 + warp * R; rb < row1; rb += kWarps * R) {
+      float acc[R][NB];
+#pragma unroll
+      for (int q = 0; q < R; ++q)
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[q][b] = 0.f;
+      for (int c = lane; c < nvec; c += kWarp) {
+        uint4 wv[R];
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+          const int row = min(rb + q, row1 - 1);
+          wv[q] = ld_stream(W2 + (size_t)row * r + (size_t)c * V);
+        }
+#pragma unroll
+        for (int q = 0; q < R; ++q)
+#pragma unroll
+          for (int b = 0; b < NB; ++b) acc[q][b] += dot_hidden<T>(wv[q], hs + (size_t)b * r, r, c);
+      }
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        const int row = rb + q;
+        bool on = false;
+        const float bias = (row < row1) ? __ldg(b2 + row) : 0.f;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const float z = warp_sum(acc[q][b]) + bias;
+          on |= (b < nb) && (z > thr);
+        }
+        if (lane == 0 && on && row < row1) atomicOr(&smask[(row >> 5) - wfirst], 1u << (row & 31));
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nwl; i += kThreads)
+    if (smask[i]) atomicOr(&mask_words[wfirst + i], smask[i]);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&hdr->done, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // ---- compaction by the last CTA: block-wide exclusive scan of popcounts ----
+  const int wpt = (n_words + kThreads - 1) / kThreads;
+  const int wbeg = min(n_words, threadIdx.x * wpt);
+  const int wend = min(n_words, wbeg + wpt);
+  int local = 0;
+  for (int w = wbeg; w < wend; ++w) local += __popc(ld_cg_u32(mask_words + w));
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < kWarp; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == kWarp - 1) s_wsum[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += s_wsum[w];
+  int off = before + incl - local;
+  for (int w = wbeg; w < wend; ++w) {
+    uint32_t m = ld_cg_u32(mask_words + w);
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      idx[off++] = w * 32 + bit;
+      m &= m - 1u;
+    }
+  }
+  if (threadIdx.x == kThreads - 1) {
+    *count = off;
+    hdr->done = 0u;
+  }
+}
+
+// ======================================================================== //
+// sparse FFN                                                               //
+// ======================================================================== //
+
+// Gate/up gather-GEMV and activation.  Warp w of the grid handles list
+// positions j = w, w + W, ...; for neuron k = idx[j] it streams the whole
+// gate and up rows once and writes a[j][b] for every token b.
+template <typename T, int NB, int U, bool REGLU>
+__global__ void __launch_bounds__(kThreads)
+    k_ffn_gu(const T *__restrict__ Wg, const T *__restrict__ Wu, const float *__restrict__ bias,
+             const T *__restrict__ x, int d, int n, int B, const int32_t *__restrict__ idx,
+             const int32_t *__restrict__ count, float *__restrict__ a, int32_t *__restrict__ err) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  T *xs = reinterpret_cast<T *>(smem_raw);
+  constexpr int V = Vec<T>::N;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
+  int cnt = n;
+  if (idx) {
+    const int c = ld_cg_i32(count);
+    if (c < 0 || c > n) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(err, kErrIndex);
+      cnt = max(0, min(c, n));
+    } else {
+      cnt = c;
+    }
+  }
+  const int nvec = d / V;
+  const int wtot = gridDim.x * kWarps;
+  const int gw = blockIdx.x * kWarps + warp;
+  for (int g0 = 0; g0 < B; g0 += NB) {
+    const int nb = min(NB, B - g0);
+    __syncthreads();
+    stage_tokens<T, NB>(xs, x, d, g0, nb);
+    __syncthreads();
+    for (int j = gw; j < cnt; j += wtot) {
+      const int k = idx ? ld_cg_i32(idx + j) : j;
+      float out[NB];
+      if ((unsigned)k >= (unsigned)n) {
+        if (lane == 0 && g0 == 0) flag_error(err, kErrIndex);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) out[b] = 0.f;
+      } else {
+        const float bk = __ldg(bias + k);
+        if constexpr (REGLU) {
+          float ag[NB], au[NB];
+#pragma unroll
+          for (int b = 0; b < NB; ++b) ag[b] = au[b] = 0.f;
+          row_dot2<T, NB, U>(Wg + (size_t)k * d, Wu + (size_t)k * d, xs, d, nvec, lane, ag, au);
+#pragma unroll
+          for (int b = 0; b < NB; ++b) out[b] = fmaxf(warp_sum(ag[b]) + bk, 0.f) * warp_sum(au[b]);
+        } else {
+          float au[NB];
+#pragma unroll
+          for (int b = 0; b < NB; ++b) au[b] = 0.f;
+          row_dot<T, NB, 2 * U>(Wu + (size_t)k * d, xs, d, nvec, lane, au);
+#pragma unroll
+          for (int b = 0; b < NB; ++b) out[b] = fmaxf(warp_sum(au[b]) + bk, 0.f);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        if (lane == b && b < nb) a[(size_t)j * B + g0 + b] = out[b];
+    }
+  }
+}
+
+// Down projection as a gather-accumulate over rows of W_down^T.  CTA (t, s)
+// owns column tile t (TW = 32 lanes x one 16-byte chunk) and the s-th slice of
+// the index list; warps split the slice, lanes own columns, so each weight row
+// chunk is one coalesced 512-byte read.  Warp partials are summed in shared
+// memory in warp order; split partials are summed in split order by the last
+// CTA of the tile (atomic ticket) -- deterministic, no float atomics.
+template <typename T, int NB, int UJ>
+__global__ void __launch_bounds__(kThreads)
+    k_ffn_down(const T *__restrict__ WdT, const float *__restrict__ a, const int32_t *__restrict__ idx,
+               const int32_t *__restrict__ count, int d, int n, int B, int S,
+               float *__restrict__ part, float *__restrict__ y, Header *__restrict__ hdr,
+               int prefetch) {
+  constexpr int V = Vec<T>::N;
+  constexpr int TW = kWarp * V;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float *red = reinterpret_cast<float *>(smem_raw);  // [kWarps][NB][TW]
+  __shared__ int s_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tile = blockIdx.x, split = blockIdx.y;
+  const int col0 = tile * TW;
+  const int col = col0 + lane * V;
+  const bool col_ok = col < d;
+  // The index list was completed two kernels earlier (the gate/up kernel
+  // waited for it before letting this grid start), so it can be read before
+  // waiting for the activations.
+  int cnt = n;
+  if (idx) cnt = max(0, min(ld_cg_i32(count), n));
+  const int js = (int)(((long long)cnt * split) / S);
+  const int je = (int)(((long long)cnt * (split + 1)) / S);
+  if (prefetch) {
+    const uint32_t bytes = (uint32_t)(min(TW, d - col0) * sizeof(T));
+    for (int j = js + threadIdx.x; j < je; j += kThreads) {
+      const int k = idx ? ld_cg_i32(idx + j) : j;
+      if ((unsigned)k < (unsigned)n) prefetch_l2(WdT + (size_t)k * d + col0, bytes);
+    }
+  }
+  pdl_wait();
+  pdl_trigger();
+  for (int g0 = 0; g0 < B; g0 += NB) {
+    const int nb = min(NB, B - g0);
+    float acc[V][NB];
+#pragma unroll
+    for (int e = 0; e < V; ++e)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) acc[e][b] = 0.f;
+    for (int j = js + warp * UJ; j < je; j += kWarps * UJ) {
+      uint4 wv[UJ];
+      float av[UJ][NB];
+#pragma unroll
+      for (int u = 0; u < UJ; ++u) {
+        const int jj = j + u;
+        int k = -1;
+        if (jj < je) k = idx ? ld_cg_i32(idx + jj) : jj;
+        const bool ok = (unsigned)k < (unsigned)n;
+        wv[u] = (ok && col_ok) ? ld_stream(WdT + (size_t)k * d + col) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+          av[u][b] = (ok && b < nb) ? ld_cg_f32(a + (size_t)jj * B + g0 + b) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < UJ; ++u) {
+        float f[V];
+        Vec<T>::to_float(wv[u], f);
+#pragma unroll
+        for (int e = 0; e < V; ++e)
+#pragma unroll
+          for (int b = 0; b < NB; ++b) acc[e][b] = fmaf(av[u][b], f[e], acc[e][b]);
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int e = 0; e < V; ++e) red[((size_t)warp * NB + b) * TW + lane * V + e] = acc[e][b];
+    __syncthreads();
+    for (int i = threadIdx.x; i < NB * TW; i += kThreads) {
+      const int b = i / TW, c = i - b * TW;
+      if (b < nb && col0 + c < d) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s += red[((size_t)w * NB + b) * TW + c];
+        if (S == 1)
+          y[(size_t)(g0 + b) * d + col0 + c] = s;
+        else
+          part[((size_t)split * B + g0 + b) * d + col0 + c] = s;
+      }
+    }
+  }
+  if (S == 1) return;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&hdr->tile_done[tile], 1u) == (unsigned)S - 1u);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int tw = min(TW, d - col0);
+  for (int i = threadIdx.x; i < B * tw; i += kThreads) {
+    const int b = i / tw, c = i - b * tw;
+    float s = 0.f;
+    for (int q = 0; q < S; ++q) s += ld_cg_f32(part + ((size_t)q * B + b) * d + col0 + c);
+    y[(size_t)b * d + col0 + c] = s;
+  }
+  if (threadIdx.x == 0) hdr->tile_done[tile] = 0u;
+}
+
+// ======================================================================== //
+// offline: activation counts and row permutation                           //
+// ======================================================================== //
+
+// counts[k] += #{t : W[k] . x_t + bias_k > 0}.  Warps own rows; the row is
+// re-read from L1/L2 for every group of NB tokens.
+template <typename T, int NB, int U>
+__global__ void __launch_bounds__(kThreads)
+    k_act_counts(const T *__restrict__ W, const float *__restrict__ bias, const T *__restrict__ x, int d,
+                 int n, int Ttok, int rpc, int64_t *__restrict__ counts) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  T *xs = reinterpret_cast<T *>(smem_raw);
+  constexpr int V = Vec<T>::N;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
+  const int row0 = blockIdx.x * rpc;
+  const int row1 = min(n, row0 + rpc);
+  const int nvec = d / V;
+  for (int rb = row0; rb < row1; rb += kWarps) {
+    const int row = rb + warp;
+    const bool ok = row < row1;
+    long long c = 0;
+    const float bk = ok ? __ldg(bias + row) : 0.f;
+    for (int g0 = 0; g0 < Ttok; g0 += NB) {
+      const int nb = min(NB, Ttok - g0);
+      __syncthreads();
+      stage_tokens<T, NB>(xs, x, d, g0, nb);
+      __syncthreads();
+      if (ok) {
+        float acc[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+        row_dot<T, NB, U>(W + (size_t)row * d, xs, d, nvec, lane, acc);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const float s = warp_sum(acc[b]) + bk;
+          c += (b < nb && s > 0.f) ? 1 : 0;
+        }
+      }
+    }
+    if (ok && lane == 0) counts[row] += c;
+  }
+}
+
+// dst row i = src row perm[i]; one CTA per row (grid-stride), widest copy
+// unit the alignment allows.
+__global__ void __launch_bounds__(kThreads)
+    k_permute_rows(const unsigned char *__restrict__ src, unsigned char *__restrict__ dst, int n_rows,
+                   long long row_bytes, const int32_t *__restrict__ perm, int unit) {
+  for (int i = blockIdx.x; i < n_rows; i += gridDim.x) {
+    const int p = __ldg(perm + i);
+    if ((unsigned)p >= (unsigned)n_rows) continue;
+    const unsigned char *s = src + (size_t)p * row_bytes;
+    unsigned char *t = dst + (size_t)i * row_bytes;
+    if (unit == 16) {
+      for (long long o = threadIdx.x; o < row_bytes / 16; o += blockDim.x)
+        reinterpret_cast<uint4 *>(t)[o] = __ldg(reinterpret_cast<const uint4 *>(s) + o);
+    } else if (unit == 4) {
+      for (long long o = threadIdx.x; o < row_bytes / 4; o += blockDim.x)
+        reinterpret_cast<uint32_t *>(t)[o] = __ldg(reinterpret_cast<const uint32_t *>(s) + o);
+    } else {
+      for (long long o = threadIdx.x; o < row_bytes; o += blockDim.x) t[o] = s[o];
+    }
+  }
+}
+
+// ======================================================================== //
+// host side                                                                //
+// ======================================================================== //
+
+struct DevCache {
+  int sms = 0;
+};
+std::mutex g_mu;
+DevCache g_dev[64];
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_dev[dev].sms == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    g_dev[dev].sms = v;
+  }
+  return g_dev[dev].sms;
+}
+
+int env_flag(const char *name, int dflt) {
+  const char *v = std::getenv(name);
+  if (!v || !*v) return dflt;
+  return std::atoi(v);
+}
+
+bool pdl_enabled() {
+  static int on = env_flag("ASFFN_PDL", 1);
+  return on != 0;
+}
+int prefetch_enabled() {
+  static int on = env_flag("ASFFN_PREFETCH", 1);
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args... args) {
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute((const void *)kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+inline size_t r256(size_t v) { return (v + 255) & ~size_t(255); }
+inline int vec_of(asf_dtype t) { return t == ASF_F16 ? 8 : 4; }
+inline int esize(asf_dtype t) { return t == ASF_F16 ? 2 : 4; }
+
+int n_words_of(int n) { return (n + 31) / 32; }
+
+// column tiles and index-list splits of the down projection
+int down_tiles(const asf_ffn *f) { return (f->d + kWarp * vec_of(f->wdtype) - 1) / (kWarp * vec_of(f->wdtype)); }
+int down_splits(const asf_ffn *f) {
+  const int ct = down_tiles(f);
+  return std::max(1, std::min(kMaxSplits, (kTargetCtas + ct - 1) / ct));
+}
+
+size_t pred_scratch(const asf_predictor *p, int B) {
+  return r256((size_t)n_words_of(p->n) * 4) + r256((size_t)B * p->r * 4);
+}
+size_t ffn_scratch(const asf_ffn *f, int B) {
+  return r256((size_t)f->n * B * 4) + r256((size_t)down_splits(f) * B * f->d * 4);
+}
+
+asf_status check_pred(const asf_predictor *p) {
+  if (!p || !p->W1 || !p->b1 || !p->W2 || !p->b2) return ASF_ERR_INVALID_ARG;
+  if (p->wdtype != ASF_F16 && p->wdtype != ASF_F32) return ASF_ERR_UNSUPPORTED;
+  if (p->d <= 0 || p->r <= 0 || p->n <= 0) return ASF_ERR_INVALID_ARG;
+  const int v = vec_of(p->wdtype);
+  if (p->d % v || p->r % v) return ASF_ERR_MISALIGNED;
+  if (!al16(p->W1) || !al16(p->W2) || !al4(p->b1) || !al4(p->b2)) return ASF_ERR_MISALIGNED;
+  if ((size_t)p->d * esize(p->wdtype) > kSmemBudget || (size_t)p->r * 4 > kSmemBudget)
+    return ASF_ERR_UNSUPPORTED;
+  return ASF_OK;
+}
+
+asf_status check_ffn(const asf_ffn *f) {
+  if (!f || !f->Wu || !f->WdT || !f->bias) return ASF_ERR_INVALID_ARG;
+  if (f->wdtype != ASF_F16 && f->wdtype != ASF_F32) return ASF_ERR_UNSUPPORTED;
+  if (f->act != ASF_ACT_RELU && f->act != ASF_ACT_REGLU) return ASF_ERR_UNSUPPORTED;
+  if (f->act == ASF_ACT_REGLU && !f->Wg) return ASF_ERR_INVALID_ARG;
+  if (f->d <= 0 || f->n <= 0) return ASF_ERR_INVALID_ARG;
+  if (f->d % vec_of(f->wdtype)) return ASF_ERR_MISALIGNED;
+  if ((size_t)f->d * esize(f->wdtype) > kSmemBudget) return ASF_ERR_UNSUPPORTED;
+  if (down_tiles(f) > kMaxTiles) return ASF_ERR_UNSUPPORTED;
+  if (!al16(f->Wu) || !al16(f->WdT) || (f->Wg && !al16(f->Wg)) || !al4(f->bias)) return ASF_ERR_MISALIGNED;
+  return ASF_OK;
+}
+
+asf_status check_ws(void *ws, size_t ws_bytes, size_t need) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return ASF_ERR_WORKSPACE;
+  if (ws_bytes < need) return ASF_ERR_WORKSPACE;
+  return ASF_OK;
+}
+
+inline asf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ASF_OK : ASF_ERR_CUDA; }
+
+// largest token group in {1, 2, 4, 8} not above B whose staging fits
+int pick_nb(int B, size_t bytes_per_token) {
+  int nb = 8;
+  while (nb > 1 && (nb > B || (size_t)nb * bytes_per_token > kSmemBudget)) nb >>= 1;
+  return nb;
+}
+
+// ---------------------------------------------------------------- predict --
+template <typename T, int NB>
+cudaError_t run_pred_l1(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, cudaStream_t st) {
+  const int sms = sm_count();
+  const int rpc = (p->r + sms - 1) / sms;
+  const int grid = (p->r + rpc - 1) / rpc;
+  const size_t smem = (size_t)NB * p->d * sizeof(T);
+  return launch(k_pred_l1<T, NB, 8>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W1, p->b1,
+                (const T *)x, p->d, p->r, B, rpc, h, mask, n_words_of(p->n), prefetch_enabled());
+}
+
+template <typename T, int NB>
+cudaError_t run_pred_l2(const asf_predictor *p, int B, float thr, const float *h, uint32_t *mask, int32_t *idx,
+                        int32_t *count, Header *hdr, cudaStream_t st) {
+  const int sms = sm_count();
+  const int rpc = (p->n + sms - 1) / sms;
+  const int grid = (p->n + rpc - 1) / rpc;
+  const size_t smem = (size_t)NB * p->r * 4 + ((size_t)rpc / 32 + 2) * 4;
+  return launch(k_pred_l2<T, NB, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W2, p->b2, h, p->r,
+                p->n, B, thr, rpc, mask, n_words_of(p->n), idx, count, hdr, prefetch_enabled());
+}
+
+template <typename T>
+asf_status predict_t(const asf_predictor *p, const void *x, int B, float thr, int32_t *idx, int32_t *count,
+                     void *ws, cudaStream_t st) {
+  unsigned char *base = static_cast<unsigned char *>(ws);
+  Header *hdr = reinterpret_cast<Header *>(base);
+  uint32_t *mask = reinterpret_cast<uint32_t *>(base + kHeaderBytes);
+  float *h = reinterpret_cast<float *>(base + kHeaderBytes + r256((size_t)n_words_of(p->n) * 4));
+  const int nb1 = pick_nb(B, (size_t)p->d * sizeof(T));
+  const int nb2 = pick_nb(B, (size_t)p->r * 4);
+  cudaError_t e;
+  switch (nb1) {
+    case 1: e = run_pred_l1<T, 1>(p, x, B, h, mask, st); break;
+    case 2: e = run_pred_l1<T, 2>(p, x, B, h, mask, st); break;
+    case 4: e = run_pred_l1<T, 4>(p, x, B, h, mask, st); break;
+    default: e = run_pred_l1<T, 8>(p, x, B, h, mask, st); break;
+  }
+  if (e != cudaSuccess) return ASF_ERR_CUDA;
+  switch (nb2) {
+    case 1: e = run_pred_l2<T, 1>(p, B, thr, h, mask, idx, count, hdr, st); break;
+    case 2: e = run_pred_l2<T, 2>(p, B, thr, h, mask, idx, count, hdr, st); break;
+    case 4: e = run_pred_l2<T, 4>(p, B, thr, h, mask, idx, count, hdr, st); break;
+    default: e = run_pred_l2<T, 8>(p, B, thr, h, mask, idx, count, hdr, st); break;
+  }
+  return cuda_status(e);
+}
+
+// ------------------------------------------------------------------- ffn --
+template <typename T, int NB>
+cudaError_t run_gu(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *a,
+                   int32_t *err, cudaStream_t st) {
+  const int grid = 2 * sm_count();
+  const size_t smem = (size_t)NB * f->d * sizeof(T);
+  if (f->act == ASF_ACT_REGLU)
+    return launch(k_ffn_gu<T, NB, 4, true>, dim3(grid), dim3(kThreads), smem, st, (const T *)f->Wg,
+                  (const T *)f->Wu, f->bias, (const T *)x, f->d, f->n, B, idx, count, a, err);
+  return launch(k_ffn_gu<T, NB, 4, false>, dim3(grid), dim3(kThreads), smem, st, (const T *)f->Wg,
+                (const T *)f->Wu, f->bias, (const T *)x, f->d, f->n, B, idx, count, a, err);
+}
+
+template <typename T, int NB>
+cudaError_t run_down(const asf_ffn *f, int B, const int32_t *idx, const int32_t *count, const float *a, float *part,
+                     float *y, Header *hdr, cudaStream_t st) {
+  constexpr int TW = kWarp * Vec<T>::N;
+  const int ct = down_tiles(f);
+  const int S = down_splits(f);
+  const size_t smem = (size_t)kWarps * NB * TW * 4;
+  return launch(k_ffn_down<T, NB, 4>, dim3(ct, S), dim3(kThreads), smem, st, (const T *)f->WdT, a, idx, count,
+                f->d, f->n, B, S, part, y, hdr, prefetch_enabled());
+}
+
+template <typename T>
+asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *y,
+                 void *ws, cudaStream_t st) {
+  unsigned char *base = static_cast<unsigned char *>(ws);
+  Header *hdr = reinterpret_cast<Header *>(base);
+  float *a = reinterpret_cast<float *>(base + kHeaderBytes);
+  float *part = reinterpret_cast<float *>(base + kHeaderBytes + r256((size_t)f->n * B * 4));
+  const int nbg = pick_nb(B, (size_t)f->d * sizeof(T));
+  cudaError_t e;
+  switch (nbg) {
+    case 1: e = run_gu<T, 1>(f, x, B, idx, count, a, &hdr->err, st); break;
+    case 2: e = run_gu<T, 2>(f, x, B, idx, count, a, &hdr->err, st); break;
+    case 4: e = run_gu<T, 4>(f, x, B, idx, count, a, &hdr->err, st); break;
+    default: e = run_gu<T, 8>(f, x, B, idx, count, a, &hdr->err, st); break;
+  }
+  if (e != cudaSuccess) return ASF_ERR_CUDA;
+  const int nbd = std::min(B >= 8 ? 8 : (B >= 4 ? 4 : (B >= 2 ? 2 : 1)), 8);
+  switch (nbd) {
+    case 1: e = run_down<T, 1>(f, B, idx, count, a, part, y, hdr, st); break;
+    case 2: e = run_down<T, 2>(f, B, idx, count, a, part, y, hdr, st); break;
+    case 4: e = run_down<T, 4>(f, B, idx, count, a, part, y, hdr, st); break;
+    default: e = run_down<T, 8>(f, B, idx, count, a, part, y, hdr, st); break;
+  }
+  return cuda_status(e);
+}
+
+template <typename T>
+asf_status counts_t(const asf_ffn *f, const void *x, int Ttok, int64_t *counts, cudaStream_t st) {
+  const int sms = sm_count();
+  const int rpc = (f->n + sms - 1) / sms;
+  const int grid = (f->n + rpc - 1) / rpc;
+  const void *W = f->act == ASF_ACT_REGLU ? f->Wg : f->Wu;
+  const int nb = pick_nb(8, (size_t)f->d * sizeof(T));
+  const size_t smem = (size_t)nb * f->d * sizeof(T);
+  cudaError_t e;
+  switch (nb) {
+    case 1: e = launch(k_act_counts<T, 1, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, f->n, Ttok, rpc, counts); break;
+    case 2: e = launch(k_act_counts<T, 2, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, f->n, Ttok, rpc, counts); break;
+    case 4: e = launch(k_act_counts<T, 4, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, f->n, Ttok, rpc, counts); break;
+    default: e = launch(k_act_counts<T, 8, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, f->n, Ttok, rpc, counts); break;
+  }
+  return cuda_status(e);
+}
+
+}  // namespace
+
+// ======================================================================== //
+// C ABI                                                                    //
+// ======================================================================== //
+extern "C" {
+
+int32_t asf_version(void) { return 100; }
+
+const char *asf_status_string(asf_status s) {
+  switch (s) {
+    case ASF_OK: return "ok";
+    case ASF_ERR_INVALID_ARG: return "invalid argument";
+    case ASF_ERR_MISALIGNED: return "misaligned pointer or size";
+    case ASF_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ASF_ERR_CUDA: return "CUDA error";
+    case ASF_ERR_DEVICE_INDEX: return "device saw an index out of range";
+    case ASF_ERR_TIMEOUT: return "bounded device wait timed out";
+    case ASF_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+  }
+  return "unknown status";
+}
+
+size_t asf_workspace_bytes(const asf_predictor *pred, const asf_ffn *ffn, int32_t max_batch) {
+  if (max_batch < 1 || max_batch > ASF_MAX_BATCH) return 0;
+  if (!pred && !ffn) return 0;
+  size_t need = 0;
+  if (pred) {
+    if (check_pred(pred) != ASF_OK) return 0;
+    need = std::max(need, pred_scratch(pred, max_batch));
+  }
+  if (ffn) {
+    if (check_ffn(ffn) != ASF_OK) return 0;
+    need = std::max(need, ffn_scratch(ffn, max_batch));
+  }
+  return kHeaderBytes + need;
+}
+
+asf_status asf_workspace_init(void *ws, size_t ws_bytes, asf_stream_t stream) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < kHeaderBytes) return ASF_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
+}
+
+asf_status asf_predict(const asf_predictor *pred, const void *x, int32_t B, float tau, int32_t *idx,
+                       int32_t *count, void *ws, size_t ws_bytes, asf_stream_t stream) {
+  asf_status s = check_pred(pred);
+  if (s != ASF_OK) return s;
+  if (!x || !idx || !count) return ASF_ERR_INVALID_ARG;
+  if (B < 1 || B > ASF_MAX_BATCH) return ASF_ERR_INVALID_ARG;
+  if (!(tau > 0.f && tau < 1.f)) return ASF_ERR_INVALID_ARG;
+  if (!al16(x) || !al4(idx) || !al4(count)) return ASF_ERR_MISALIGNED;
+  s = check_ws(ws, ws_bytes, kHeaderBytes + pred_scratch(pred, B));
+  if (s != ASF_OK) return s;
+  // sigmoid(z) > tau  <=>  z > log(tau / (1 - tau)), evaluated once in double
+  const float thr = (float)std::log((double)tau / (1.0 - (double)tau));
+  if (pred->wdtype == ASF_F16)
+    return predict_t<__half>(pred, x, B, thr, idx, count, ws, (cudaStream_t)stream);
+  return predict_t<float>(pred, x, B, thr, idx, count, ws, (cudaStream_t)stream);
+}
+
+asf_status asf_sparse_ffn(const asf_ffn *ffn, const void *x, int32_t B, const int32_t *idx, const int32_t *count,
+                          float *y, void *ws, size_t ws_bytes, asf_stream_t stream) {
+  asf_status s = check_ffn(ffn);
+  if (s != ASF_OK) return s;
+  if (!x || !idx || !count || !y) return ASF_ERR_INVALID_ARG;
+  if (B < 1 || B > ASF_MAX_BATCH) return ASF_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(y) || !al4(idx) || !al4(count)) return ASF_ERR_MISALIGNED;
+  s = check_ws(ws, ws_bytes, kHeaderBytes + ffn_scratch(ffn, B));
+  if (s != ASF_OK) return s;
+  if (ffn->wdtype == ASF_F16) return ffn_t<__half>(ffn, x, B, idx, count, y, ws, (cudaStream_t)stream);
+  return ffn_t<float>(ffn, x, B, idx, count, y, ws, (cudaStream_t)stream);
+}
+
+asf_status asf_dense_ffn(const asf_ffn *ffn, const void *x, int32_t B, float *y, void *ws, size_t ws_bytes,
+                         asf_stream_t stream) {
+  asf_status s = check_ffn(ffn);
+  if (s != ASF_OK) return s;
+  if (!x || !y) return ASF_ERR_INVALID_ARG;
+  if (B < 1 || B > ASF_MAX_BATCH) return ASF_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(y)) return ASF_ERR_MISALIGNED;
+  s = check_ws(ws, ws_bytes, kHeaderBytes + ffn_scratch(ffn, B));
+  if (s != ASF_OK) return s;
+  if (ffn->wdtype == ASF_F16) return ffn_t<__half>(ffn, x, B, nullptr, nullptr, y, ws, (cudaStream_t)stream);
+  return ffn_t<float>(ffn, x, B, nullptr, nullptr, y, ws, (cudaStream_t)stream);
+}
+
+asf_status asf_activation_counts(const asf_ffn *ffn, const void *x, int32_t T, int64_t *counts, void *ws,
+                                 size_t ws_bytes, asf_stream_t stream) {
+  asf_status s = check_ffn(ffn);
+  if (s != ASF_OK) return s;
+  if (!x || !counts || T < 0) return ASF_ERR_INVALID_ARG;
+  if (!al16(x) || (reinterpret_cast<uintptr_t>(counts) & 7u)) return ASF_ERR_MISALIGNED;
+  s = check_ws(ws, ws_bytes, kHeaderBytes);
+  if (s != ASF_OK) return s;
+  if (T == 0) return ASF_OK;
+  if (ffn->wdtype == ASF_F16) return counts_t<__half>(ffn, x, T, counts, (cudaStream_t)stream);
+  return counts_t<float>(ffn, x, T, counts, (cudaStream_t)stream);
+}
+
+asf_status asf_hot_permutation(const int64_t *counts, int32_t n, int32_t *perm_out) {
+  if (!counts || !perm_out || n < 0) return ASF_ERR_INVALID_ARG;
+  std::vector<int32_t> order((size_t)n);
+  for (int32_t i = 0; i < n; ++i) order[(size_t)i] = i;
+  std::stable_sort(order.begin(), order.end(),
+                   [counts](int32_t a, int32_t b) { return counts[a] > counts[b]; });
+  std::memcpy(perm_out, order.data(), (size_t)n * sizeof(int32_t));
+  return ASF_OK;
+}
+
+asf_status asf_permute_rows(const void *src, void *dst, int32_t n_rows, int64_t row_bytes, const int32_t *perm,
+                            asf_stream_t stream) {
+  if (!src || !dst || !perm || n_rows < 0 || row_bytes <= 0) return ASF_ERR_INVALID_ARG;
+  if (src == dst) return ASF_ERR_INVALID_ARG;
+  if (!al4(perm)) return ASF_ERR_MISALIGNED;
+  if (n_rows == 0) return ASF_OK;
+  int unit = 1;
+  if (row_bytes % 16 == 0 && al16(src) && al16(dst))
+    unit = 16;
+  else if (row_bytes % 4 == 0 && al4(src) && al4(dst))
+    unit = 4;
+  const int grid = std::min(n_rows, 8 * sm_count());
+  return cuda_status(launch(k_permute_rows, dim3(grid), dim3(kThreads), 0, (cudaStream_t)stream,
+                            (const unsigned char *)src, (unsigned char *)dst, (int)n_rows, (long long)row_bytes,
+                            perm, unit));
+}
+
+asf_status asf_read_error(void *ws, int32_t *host_out, asf_stream_t stream) {
+  if (!ws || !host_out) return ASF_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return ASF_ERR_WORKSPACE;
+  int32_t v = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return ASF_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess) return ASF_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ASF_ERR_CUDA;
+  int32_t out = ASF_OK;
+  if (v & kErrIndex)
+    out = ASF_ERR_DEVICE_INDEX;
+  else if (v & kErrTimeout)
+    out = ASF_ERR_TIMEOUT;
+  *host_out = out;
+  return ASF_OK;
+}
+
+}  // extern "C"

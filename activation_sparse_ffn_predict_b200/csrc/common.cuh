@@ -1,0 +1,134 @@
+// Device helpers shared by the asffn kernels (sm_100a).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace asf {
+
+constexpr int kWarp = 32;
+
+// Bits of the device error word (workspace offset 0).
+constexpr int kErrIndex = 1;    // idx outside [0, n) or count outside [0, n]
+constexpr int kErrTimeout = 2;  // a bounded wait gave up
+
+// Workspace header: error word, compaction ticket, per-column-tile tickets.
+constexpr size_t kHeaderBytes = 4096;
+constexpr int kMaxTiles = 960;  // ticket slots for the down-projection reduction
+struct Header {
+  int32_t err;
+  uint32_t done;
+  uint32_t pad[14];
+  uint32_t tile_done[kMaxTiles];
+};
+static_assert(sizeof(Header) <= kHeaderBytes, "header too large");
+
+// ---------------------------------------------------------------- PTX --
+// Streaming 16-byte load of read-only weights: skip L1 allocation.
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+// Load of data another kernel (or CTA) produced: served from L2, never L1.
+__device__ __forceinline__ int ld_cg_i32(const int32_t *p) { return __ldcg(p); }
+__device__ __forceinline__ float ld_cg_f32(const float *p) { return __ldcg(p); }
+__device__ __forceinline__ uint32_t ld_cg_u32(const uint32_t *p) { return __ldcg(p); }
+
+// Programmatic dependent launch: wait for the preceding grid's memory, and
+// allow the next grid in the stream to start its prologue.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Bulk prefetch of a contiguous range into L2 (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void flag_error(int32_t *err, int bit) {
+  if (err) atomicOr(err, bit);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ------------------------------------------------------- element types --
+// Vec<T>: one 16-byte chunk of weights holds N elements of T.
+template <typename T> struct Vec;
+
+template <> struct Vec<float> {
+  static constexpr int N = 4;
+  // acc + sum_i w_i * x_i, x in the same 16-byte layout
+  __device__ __forceinline__ static float dot(uint4 w, uint4 x, float acc) {
+    acc = fmaf(__uint_as_float(w.x), __uint_as_float(x.x), acc);
+    acc = fmaf(__uint_as_float(w.y), __uint_as_float(x.y), acc);
+    acc = fmaf(__uint_as_float(w.z), __uint_as_float(x.z), acc);
+    acc = fmaf(__uint_as_float(w.w), __uint_as_float(x.w), acc);
+    return acc;
+  }
+  // acc + sum_i w_i * x_i with x as N floats
+  __device__ __forceinline__ static float dotf(uint4 w, const float *x, float acc) {
+    const float4 a = *reinterpret_cast<const float4 *>(x);
+    acc = fmaf(__uint_as_float(w.x), a.x, acc);
+    acc = fmaf(__uint_as_float(w.y), a.y, acc);
+    acc = fmaf(__uint_as_float(w.z), a.z, acc);
+    acc = fmaf(__uint_as_float(w.w), a.w, acc);
+    return acc;
+  }
+  __device__ __forceinline__ static void to_float(uint4 w, float (&f)[4]) {
+    f[0] = __uint_as_float(w.x);
+    f[1] = __uint_as_float(w.y);
+    f[2] = __uint_as_float(w.z);
+    f[3] = __uint_as_float(w.w);
+  }
+};
+
+template <> struct Vec<__half> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static float2 h2f(uint32_t u) {
+    __half2 h = *reinterpret_cast<__half2 *>(&u);
+    return __half22float2(h);
+  }
+  __device__ __forceinline__ static float dot(uint4 w, uint4 x, float acc) {
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 a = h2f(wv[i]);
+      const float2 b = h2f(xv[i]);
+      acc = fmaf(a.x, b.x, acc);
+      acc = fmaf(a.y, b.y, acc);
+    }
+    return acc;
+  }
+  // x: 8 floats split in two 4-float planes at x0 and x1
+  __device__ __forceinline__ static float dotf2(uint4 w, const float *x0, const float *x1,
+                                                float acc) {
+    const float4 a = *reinterpret_cast<const float4 *>(x0);
+    const float4 b = *reinterpret_cast<const float4 *>(x1);
+    float2 p;
+    p = h2f(w.x); acc = fmaf(p.x, a.x, acc); acc = fmaf(p.y, a.y, acc);
+    p = h2f(w.y); acc = fmaf(p.x, a.z, acc); acc = fmaf(p.y, a.w, acc);
+    p = h2f(w.z); acc = fmaf(p.x, b.x, acc); acc = fmaf(p.y, b.y, acc);
+    p = h2f(w.w); acc = fmaf(p.x, b.z, acc); acc = fmaf(p.y, b.w, acc);
+    return acc;
+  }
+  __device__ __forceinline__ static void to_float(uint4 w, float (&f)[8]) {
+    float2 p;
+    p = h2f(w.x); f[0] = p.x; f[1] = p.y;
+    p = h2f(w.y); f[2] = p.x; f[3] = p.y;
+    p = h2f(w.z); f[4] = p.x; f[5] = p.y;
+    p = h2f(w.w); f[6] = p.x; f[7] = p.y;
+  }
+};
+
+}  // namespace asf

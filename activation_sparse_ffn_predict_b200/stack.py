@@ -1,0 +1,87 @@
+"""A decode step over a stack of FFN layers: predictor then sparse FFN per layer.
+
+One step takes the B tokens' FFN inputs for every layer (``x[l]``), runs
+asf_predict and asf_sparse_ffn for l = 0..L-1 in order on one stream, and
+leaves y[l], idx[l], count[l] on the device.  The launch sequence is captured
+once into a CUDA graph; kernels inside it overlap through programmatic
+dependent launch (each waits for its predecessor before reading its inputs).
+"""
+from __future__ import annotations
+
+from typing import List, Optional, Sequence
+
+import torch
+
+from .api import (FFN, Predictor, Workspace, asf_dense_ffn, asf_predict, asf_sparse_ffn)
+
+
+class LayerStack:
+    def __init__(self, preds: Sequence[Optional[Predictor]], ffns: Sequence[FFN], batch: int,
+                 tau: float = 0.5, mode: str = "predict", device=None):
+        """mode: "predict" (predictor + sparse FFN), "sparse" (sparse FFN over
+        caller-filled idx/count), or "dense" (all neurons)."""
+        if mode not in ("predict", "sparse", "dense"):
+            raise ValueError("mode must be predict, sparse or dense")
+        self.preds = list(preds)
+        self.ffns = list(ffns)
+        self.L = len(self.ffns)
+        self.B = int(batch)
+        self.tau = float(tau)
+        self.mode = mode
+        f0 = self.ffns[0]
+        dev = device if device is not None else f0.tensors[1].device
+        self.d, self.n, self.dtype = f0.d, f0.n, f0.dtype
+        self.x = torch.zeros(self.L, self.B, self.d, dtype=self.dtype, device=dev)
+        self.y = torch.zeros(self.L, self.B, self.d, dtype=torch.float32, device=dev)
+        self.idx = torch.zeros(self.L, self.n, dtype=torch.int32, device=dev)
+        self.count = torch.zeros(self.L, dtype=torch.int32, device=dev)
+        p0 = self.preds[0] if (self.preds and mode == "predict") else None
+        self.ws = Workspace(p0, f0, self.B, device=dev)
+        self.graph: Optional[torch.cuda.CUDAGraph] = None
+
+    def launches_per_step(self) -> int:
+        """Kernels this library launches per step."""
+        return self.L * (4 if self.mode == "predict" else 2)
+
+    def enqueue(self, stream=None) -> None:
+        for l in range(self.L):
+            x, y = self.x[l], self.y[l]
+            if self.mode == "dense":
+                asf_dense_ffn(self.ffns[l], x, y, self.ws, stream)
+                continue
+            cnt = self.count[l:l + 1]
+            if self.mode == "predict":
+                asf_predict(self.preds[l], x, self.tau, self.idx[l], cnt, self.ws, stream)
+            asf_sparse_ffn(self.ffns[l], x, self.idx[l], cnt, y, self.ws, stream)
+
+    def capture(self, warmup: int = 2) -> None:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for _ in range(warmup):
+                self.enqueue()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.enqueue()
+        torch.cuda.synchronize()
+        self.graph = g
+
+    def step(self) -> None:
+        if self.graph is None:
+            self.enqueue()
+        else:
+            self.graph.replay()
+
+    def release(self) -> None:
+        self.graph = None
+
+
+def build_layers(weights: List, device) -> tuple:
+    """Predictor and FFN descriptors for a list of ``synthetic.LayerWeights`` on ``device``."""
+    preds, ffns = [], []
+    for w in weights:
+        preds.append(Predictor(w.W1, w.b1, w.W2, w.b2))
+        ffns.append(FFN(w.act, w.Wg, w.Wu, w.WdT, w.bias))
+    return preds, ffns

@@ -1,0 +1,167 @@
+/*
+ * asffn.h -- C ABI of libasffn.so: activation-sparse FFN decode on B200 (sm_100a).
+ *
+ * The operations follow the problem statement of the pages on PowerInfer-style
+ * neuron-level sparse inference:
+ *   - predict(x) -> active index list: the online neuron predictor
+ *     ("PowerInfer Guide: Exploiting Activation Sparsity for LLM AI", section 3
+ *     "Adaptive Online Neuron Predictors", predictor equation and the Step 2
+ *     predictor module), read as the 2-layer MLP of the "PowerInfer_x64" page
+ *     ("Prediction and Caching"): h = ReLU(W1 x + b1), z = W2 h + b2,
+ *     neuron k active iff sigmoid(z_k) > tau (strict), i.e. z_k > logit(tau).
+ *   - sparse_ffn(x, idx) -> y: the neuron-aware sparse operator (PowerInfer
+ *     Guide, section 4 "Neuron-Aware Sparse GPU Operators", and the FFN
+ *     equation of "The Hidden Inefficiency") evaluated only for listed neurons.
+ *   - activation counts + hot permutation: the offline profiler and hot/cold
+ *     split (PowerInfer Guide, Step 1), used to store hot rows first.
+ *
+ * Conventions shared by every call:
+ *   - All pointers named "device" are CUDA device pointers owned by the caller;
+ *     the library never allocates or frees device memory and never keeps a
+ *     pointer after a call returns (the descriptor structs are read at call
+ *     time only).
+ *   - Calls that take a stream enqueue work on it and return without
+ *     synchronising (except asf_read_error).  Launch failures return
+ *     ASF_ERR_CUDA; no call terminates the process.
+ *   - Arguments are validated on the host before any launch; a call that
+ *     returns an error has enqueued nothing.
+ *   - Checks that need device data (an index outside [0, n), count > n) cannot
+ *     be done on the host: the kernel skips the offending item and records the
+ *     fault in the workspace error word, read with asf_read_error.
+ *   - Weights, x and y must be 16-byte aligned; d and r must be multiples of 8
+ *     (fp16) or 4 (fp32).  x has the weight dtype; y is always fp32.
+ *   - Accumulation is fp32 throughout.
+ */
+#ifndef ASFFN_H
+#define ASFFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ASF_API __attribute__((visibility("default")))
+#else
+#define ASF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *asf_stream_t;
+
+typedef enum {
+  ASF_OK = 0,
+  ASF_ERR_INVALID_ARG = 1,  /* null pointer, bad size, tau outside (0,1), ... */
+  ASF_ERR_MISALIGNED = 2,   /* a pointer or row length breaks the alignment rule */
+  ASF_ERR_UNSUPPORTED = 3,  /* dtype/activation/batch combination not built */
+  ASF_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  ASF_ERR_DEVICE_INDEX = 5, /* device saw idx outside [0, n) or count > n */
+  ASF_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up */
+  ASF_ERR_WORKSPACE = 7     /* workspace missing, misaligned or too small */
+} asf_status;
+
+typedef enum { ASF_F32 = 0, ASF_F16 = 1 } asf_dtype;
+
+/* ASF_ACT_RELU : y = W_down ReLU(W_up x + b)                  (up + down)
+ * ASF_ACT_REGLU: y = W_down (ReLU(W_gate x + b) * (W_up x))   (gate, up, down) */
+typedef enum { ASF_ACT_RELU = 0, ASF_ACT_REGLU = 1 } asf_act;
+
+#define ASF_MAX_BATCH 32
+
+/* Two-layer predictor, borrowed device pointers.  Row-major. */
+typedef struct {
+  int32_t d;          /* input width (hidden size) */
+  int32_t r;          /* predictor hidden width */
+  int32_t n;          /* number of FFN neurons (d_ffn) */
+  asf_dtype wdtype;   /* dtype of W1, W2 and of x */
+  const void *W1;     /* [r][d] */
+  const float *b1;    /* [r] */
+  const void *W2;     /* [n][r] */
+  const float *b2;    /* [n] */
+} asf_predictor;
+
+/* One FFN layer, borrowed device pointers.  Row k of every matrix belongs to
+ * neuron k in storage order (after any hot permutation). */
+typedef struct {
+  int32_t d;          /* hidden size */
+  int32_t n;          /* number of neurons */
+  asf_dtype wdtype;   /* dtype of Wg, Wu, WdT and of x */
+  asf_act act;
+  const void *Wg;     /* [n][d] gate rows (REGLU), NULL for RELU */
+  const void *Wu;     /* [n][d] up rows */
+  const void *WdT;    /* [n][d] W_down transposed: row k = column k of W_down */
+  const float *bias;  /* [n] bias of the ReLU input: gate (REGLU) or up (RELU) */
+} asf_ffn;
+
+/* Bytes of device workspace needed by asf_predict / asf_sparse_ffn /
+ * asf_dense_ffn / asf_activation_counts for batches up to max_batch.  Either
+ * descriptor may be NULL.  Returns 0 on invalid arguments. */
+ASF_API size_t asf_workspace_bytes(const asf_predictor *pred, const asf_ffn *ffn, int32_t max_batch);
+
+/* Zero a freshly allocated workspace (256-byte aligned device buffer).  Must be
+ * called once before first use; afterwards every call leaves the workspace's
+ * counters at zero again.  One workspace serves one stream at a time. */
+ASF_API asf_status asf_workspace_init(void *ws, size_t ws_bytes, asf_stream_t stream);
+
+/* Online predictor for B tokens (1 <= B <= ASF_MAX_BATCH).
+ *   x     device [B][d], wdtype
+ *   tau   threshold on sigmoid(z), 0 < tau < 1
+ *   idx   device int32 [n]: on completion idx[0..count) holds the ascending
+ *         storage indices of the neurons predicted active for at least one of
+ *         the B tokens (the union); entries past count are left untouched
+ *   count device int32 [1]
+ * Stays on the device: no host synchronisation. */
+ASF_API asf_status asf_predict(const asf_predictor *pred, const void *x, int32_t B, float tau,
+                       int32_t *idx, int32_t *count, void *ws, size_t ws_bytes,
+                       asf_stream_t stream);
+
+/* Sparse FFN over an index list, every token over the same list.
+ *   x     device [B][d], wdtype
+ *   idx   device int32 [n]; the first *count entries are used (any order,
+ *         duplicates are summed twice); entries outside [0, n) are skipped and
+ *         flagged
+ *   count device int32 [1], 0 <= *count <= n (larger is clamped and flagged)
+ *   y     device fp32 [B][d], overwritten: y_b = sum_j a_{idx_j, b} WdT[idx_j]
+ *         with a = ReLU(gate + bias) * up  (REGLU)  or  ReLU(up + bias)  (RELU) */
+ASF_API asf_status asf_sparse_ffn(const asf_ffn *ffn, const void *x, int32_t B, const int32_t *idx,
+                          const int32_t *count, float *y, void *ws, size_t ws_bytes,
+                          asf_stream_t stream);
+
+/* Dense FFN over all n neurons (the unsparsified reference, same kernels with an
+ * implicit identity index list).  Arguments as asf_sparse_ffn. */
+ASF_API asf_status asf_dense_ffn(const asf_ffn *ffn, const void *x, int32_t B, float *y, void *ws,
+                         size_t ws_bytes, asf_stream_t stream);
+
+/* Offline profiler: counts[k] += number of the T tokens of x (device [T][d])
+ * whose ReLU input (gate + bias for REGLU, up + bias for RELU) is > 0.
+ * counts: device int64 [n], accumulated so calibration can be chunked. */
+ASF_API asf_status asf_activation_counts(const asf_ffn *ffn, const void *x, int32_t T, int64_t *counts,
+                                 void *ws, size_t ws_bytes, asf_stream_t stream);
+
+/* Host-side, synchronous: perm = neuron ids in descending count order, equal
+ * counts in ascending id order.  counts: host int64 [n]; perm_out: host int32 [n]. */
+ASF_API asf_status asf_hot_permutation(const int64_t *counts, int32_t n, int32_t *perm_out);
+
+/* Row gather on the device: dst row i = src row perm[i], for i < n_rows.
+ * src, dst: device [n_rows][row_bytes], distinct buffers; perm: device int32
+ * [n_rows] with values in [0, n_rows) (out-of-range rows are skipped). */
+ASF_API asf_status asf_permute_rows(const void *src, void *dst, int32_t n_rows, int64_t row_bytes,
+                            const int32_t *perm, asf_stream_t stream);
+
+/* Wait for the stream, then return (in *host_out) and clear the device error
+ * word: 0, or the asf_status of the first device-side fault recorded. */
+ASF_API asf_status asf_read_error(void *ws, int32_t *host_out, asf_stream_t stream);
+
+/* Static description of a status code. */
+ASF_API const char *asf_status_string(asf_status s);
+
+/* ABI version: major * 100 + minor. */
+ASF_API int32_t asf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ASFFN_H */

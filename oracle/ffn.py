@@ -110,14 +110,13 @@ def relu_input(act: str, Wg, Wu, bias, x, idx=None) -> np.ndarray:
     ReGLU: W_gate[k] . x + b_k;  plain ReLU FFN: W_up[k] . x + b_k.
     """
     X = _tokens(x)
-    W = Wg if act == "reglu" else Wu
-    W = _f64(W)
-    b = _f64(bias)
+    W = np.asarray(Wg if act == "reglu" else Wu)
+    b = np.asarray(bias)
     if idx is not None:
         idx = np.asarray(idx, dtype=np.int64)
         W = W[idx]
         b = b[idx]
-    return X @ W.T + b[None, :]
+    return X @ _f64(W).T + _f64(b)[None, :]
 
 
 def activations(act: str, Wg, Wu, bias, x, idx) -> np.ndarray:
@@ -130,7 +129,7 @@ def activations(act: str, Wg, Wu, bias, x, idx) -> np.ndarray:
     idx = np.asarray(idx, dtype=np.int64)
     pre = relu_input(act, Wg, Wu, bias, X, idx)
     if act == "reglu":
-        up = X @ _f64(Wu)[idx].T
+        up = X @ _f64(np.asarray(Wu)[idx]).T
         return np.maximum(pre, 0.0) * up
     if act == "relu":
         return np.maximum(pre, 0.0)
@@ -147,7 +146,7 @@ def sparse_ffn(act: str, Wg, Wu, WdT, bias, x, idx) -> np.ndarray:
     if idx.size == 0:
         return np.zeros((X.shape[0], np.asarray(WdT).shape[1]), dtype=np.float64)
     a = activations(act, Wg, Wu, bias, X, idx)
-    return a @ _f64(WdT)[idx]
+    return a @ _f64(np.asarray(WdT)[idx])
 
 
 def dense_ffn(act: str, Wg, Wu, WdT, bias, x) -> np.ndarray:

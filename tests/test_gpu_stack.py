@@ -1,0 +1,55 @@
+"""The layer stack as the benchmark runs it (CUDA graph, programmatic dependent
+launch between kernels) matches the oracle layer by layer."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synthetic as S
+from tests.gpu_util import ensure_built
+from tests.helpers import TOL, condition_b2, rel_err
+
+import activation_sparse_ffn_predict_b200 as A
+from activation_sparse_ffn_predict_b200.stack import LayerStack, build_layers
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("B", [1, 4])
+@pytest.mark.parametrize("mode", ["predict", "dense"])
+def test_graph_stack_matches_oracle(B, mode):
+    ensure_built()
+    cfg = S.get("llama2_7b_reglu").with_(d=1024, n=2752, r=128, layers=3)
+    tokens = 3 * B
+    hosts, devs, xs = [], [], []
+    for l in range(cfg.layers):
+        w = S.layer_weights(cfg, l)
+        X = S.layer_tokens(cfg, l, tokens)
+        h = w.numpy()
+        h["b2"] = condition_b2(h["W1"], h["b1"], h["W2"], h["b2"], X.numpy(), cfg.tau)
+        w.b2 = torch.from_numpy(h["b2"])
+        hosts.append(h)
+        devs.append(w.to("cuda"))
+        xs.append(X)
+    preds, ffns = build_layers(devs, "cuda")
+    st = LayerStack(preds, ffns, B, cfg.tau, mode=mode)
+    st.capture()
+    for step in range(3):
+        rows = slice(step * B, step * B + B)
+        for l in range(cfg.layers):
+            st.x[l].copy_(xs[l][rows].cuda())
+        st.step()
+        torch.cuda.synchronize()
+        for l in range(cfg.layers):
+            h = hosts[l]
+            Xl = xs[l][rows].numpy()
+            if mode == "dense":
+                ref = O.dense_ffn(h["act"], h["Wg"], h["Wu"], h["WdT"], h["bias"], Xl)
+            else:
+                idx = O.predict(h["W1"], h["b1"], h["W2"], h["b2"], Xl, cfg.tau)[0]
+                c = int(st.count[l].item())
+                np.testing.assert_array_equal(st.idx[l, :c].cpu().numpy(), idx)
+                ref = O.sparse_ffn(h["act"], h["Wg"], h["Wu"], h["WdT"], h["bias"], Xl, idx)
+            assert rel_err(st.y[l].cpu().numpy(), ref) <= TOL[cfg.dtype]
+    assert A.asf_read_error(st.ws) == 0
+    st.release()

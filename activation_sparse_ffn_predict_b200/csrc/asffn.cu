@@ -22,6 +22,7 @@
 // Consecutive kernels overlap through programmatic dependent launch: each
 // kernel may prefetch its weights into L2 before waiting for its inputs.
 
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -29,7 +30,9 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "asffn.h"
@@ -44,6 +47,13 @@ constexpr int kWarps = kThreads / kWarp;
 constexpr int kMaxSplits = 64;        // max CTAs summing into one column tile
 constexpr int kTargetCtas = 296;      // 2 CTAs on each of the 148 SMs
 constexpr size_t kSmemBudget = 96 * 1024;
+constexpr int kFusedWarps = 8;        // consumer warps of the fused sparse FFN
+constexpr int kCluster = 8;           // CTAs per cluster (DSMEM reduction of y)
+constexpr int kMaxClusters = 32;      // partial-sum slots per column block
+constexpr size_t kFusedSmemDefault = 160 * 1024;
+constexpr uint64_t kWaitNs = 200ull * 1000 * 1000;  // bound on any mbarrier wait
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ======================================================================== //
 // shared building blocks                                                   //
@@ -51,32 +61,29 @@ constexpr size_t kSmemBudget = 96 * 1024;
 
 // Dot products of one weight row with NB activation vectors held in shared
 // memory in the weight's own 16-byte chunk layout.  Lane l handles chunks
-// l, l+32, ...; U chunks are in flight per lane.  Returns lane partial sums.
+// l, l+32, ...; U chunks per lane are loaded before any is used (predicated
+// at the row end), so a warp keeps U x 512 bytes in flight.
 template <typename T, int NB, int U>
 __device__ __forceinline__ void row_dot(const T *__restrict__ w, const T *xs, int xs_stride,
                                         int nvec, int lane, float (&acc)[NB]) {
   constexpr int V = Vec<T>::N;
-  int c = lane;
-  for (; c + (U - 1) * kWarp < nvec; c += U * kWarp) {
+  for (int c0 = lane; c0 < nvec; c0 += U * kWarp) {
     uint4 wv[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) wv[u] = ld_stream(w + (size_t)(c + u * kWarp) * V);
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * kWarp;
+      wv[u] = c < nvec ? ld_stream(w + (size_t)c * V) : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * kWarp;
+      if (c < nvec) {
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const uint4 xv =
-            *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)(c + u * kWarp) * V);
-        acc[b] = Vec<T>::dot(wv[u], xv, acc[b]);
+        for (int b = 0; b < NB; ++b) {
+          const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)c * V);
+          acc[b] = Vec<T>::dot(wv[u], xv, acc[b]);
+        }
       }
-    }
-  }
-  for (; c < nvec; c += kWarp) {
-    const uint4 wv = ld_stream(w + (size_t)c * V);
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)c * V);
-      acc[b] = Vec<T>::dot(wv, xv, acc[b]);
     }
   }
 }
@@ -87,33 +94,26 @@ __device__ __forceinline__ void row_dot2(const T *__restrict__ w0, const T *__re
                                          const T *xs, int xs_stride, int nvec, int lane,
                                          float (&acc0)[NB], float (&acc1)[NB]) {
   constexpr int V = Vec<T>::N;
-  int c = lane;
-  for (; c + (U - 1) * kWarp < nvec; c += U * kWarp) {
+  for (int c0 = lane; c0 < nvec; c0 += U * kWarp) {
     uint4 wa[U], wb[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      wa[u] = ld_stream(w0 + (size_t)(c + u * kWarp) * V);
-      wb[u] = ld_stream(w1 + (size_t)(c + u * kWarp) * V);
+      const int c = c0 + u * kWarp;
+      const bool in = c < nvec;
+      wa[u] = in ? ld_stream(w0 + (size_t)c * V) : make_uint4(0u, 0u, 0u, 0u);
+      wb[u] = in ? ld_stream(w1 + (size_t)c * V) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * kWarp;
+      if (c < nvec) {
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const uint4 xv =
-            *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)(c + u * kWarp) * V);
-        acc0[b] = Vec<T>::dot(wa[u], xv, acc0[b]);
-        acc1[b] = Vec<T>::dot(wb[u], xv, acc1[b]);
+        for (int b = 0; b < NB; ++b) {
+          const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)c * V);
+          acc0[b] = Vec<T>::dot(wa[u], xv, acc0[b]);
+          acc1[b] = Vec<T>::dot(wb[u], xv, acc1[b]);
+        }
       }
-    }
-  }
-  for (; c < nvec; c += kWarp) {
-    const uint4 wa = ld_stream(w0 + (size_t)c * V);
-    const uint4 wb = ld_stream(w1 + (size_t)c * V);
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)b * xs_stride + (size_t)c * V);
-      acc0[b] = Vec<T>::dot(wa, xv, acc0[b]);
-      acc1[b] = Vec<T>::dot(wb, xv, acc1[b]);
     }
   }
 }
@@ -154,16 +154,24 @@ template <typename T, int NB, int U>
 __global__ void __launch_bounds__(kThreads)
     k_pred_l1(const T *__restrict__ W1, const float *__restrict__ b1, const T *__restrict__ x, int d,
               int r, int B, int rpc, float *__restrict__ h, uint32_t *__restrict__ mask_words,
-              int n_words, int prefetch) {
+              int n_words, const T *__restrict__ W2, int n, int prefetch) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   T *xs = reinterpret_cast<T *>(smem_raw);
   constexpr int V = Vec<T>::N;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row0 = blockIdx.x * rpc;
   const int row1 = min(r, row0 + rpc);
-  if (prefetch && row0 < row1) prefetch_range(W1 + (size_t)row0 * d, (size_t)(row1 - row0) * d * sizeof(T));
-  pdl_wait();
+  if (prefetch) {
+    // this CTA's W1 rows, and its share of W2 for the second predictor layer:
+    // both stream into L2 while the previous kernel is still running
+    if (row0 < row1) prefetch_range(W1 + (size_t)row0 * d, (size_t)(row1 - row0) * d * sizeof(T));
+    const int w0 = (int)(((long long)n * blockIdx.x) / gridDim.x);
+    const int w1 = (int)(((long long)n * (blockIdx.x + 1)) / gridDim.x);
+    if (w0 < w1) prefetch_range(W2 + (size_t)w0 * r, (size_t)(w1 - w0) * r * sizeof(T));
+  }
+  // The next kernel reads only weights before it waits on this one.
   pdl_trigger();
+  pdl_wait();
   for (int w = blockIdx.x * kThreads + threadIdx.x; w < n_words; w += gridDim.x * kThreads)
     mask_words[w] = 0u;
   const int nvec = d / V;
@@ -218,7 +226,7 @@ __device__ __forceinline__ float dot_hidden(uint4 w, const float *hsb, int r, in
 // each warp computes R rows at a time.  Bits of rows predicted active for any
 // token are OR-ed into the global union mask; the last CTA to finish (atomic
 // ticket, no waiting) turns the mask into the ascending index list.
-template <typename T, int NB, int R>
+template <typename T, int NB, int R, int UC>
 __global__ void __launch_bounds__(kThreads)
     k_pred_l2(const T *__restrict__ W2, const float *__restrict__ b2, const float *__restrict__ h,
               int r, int n, int B, float thr, int rpc, uint32_t *__restrict__ mask_words, int n_words,
@@ -237,8 +245,8 @@ __global__ void __launch_bounds__(kThreads)
   const int wfirst = row0 >> 5;
   const int nwl = (row0 < row1) ? (((row1 - 1) >> 5) - wfirst + 1) : 0;
   for (int i = threadIdx.x; i < nwl; i += kThreads) smask[i] = 0u;
-  pdl_wait();
   pdl_trigger();
+  pdl_wait();
   const int nvec = r / V;
   for (int g0 = 0; g0 < B; g0 += NB) {
     const int nb = min(NB, B - g0);
@@ -251,17 +259,27 @@ __global__ void __launch_bounds__(kThreads)
       for (int q = 0; q < R; ++q)
 #pragma unroll
         for (int b = 0; b < NB; ++b) acc[q][b] = 0.f;
-      for (int c = lane; c < nvec; c += kWarp) {
-        uint4 wv[R];
+      for (int c0 = lane; c0 < nvec; c0 += UC * kWarp) {
+        uint4 wv[R][UC];
 #pragma unroll
         for (int q = 0; q < R; ++q) {
           const int row = min(rb + q, row1 - 1);
-          wv[q] = ld_stream(W2 + (size_t)row * r + (size_t)c * V);
+#pragma unroll
+          for (int u = 0; u < UC; ++u) {
+            const int c = c0 + u * kWarp;
+            wv[q][u] = c < nvec ? ld_stream(W2 + (size_t)row * r + (size_t)c * V) : make_uint4(0u, 0u, 0u, 0u);
+          }
         }
 #pragma unroll
-        for (int q = 0; q < R; ++q)
+        for (int u = 0; u < UC; ++u) {
+          const int c = c0 + u * kWarp;
+          if (c < nvec) {
 #pragma unroll
-          for (int b = 0; b < NB; ++b) acc[q][b] += dot_hidden<T>(wv[q], hs + (size_t)b * r, r, c);
+            for (int q = 0; q < R; ++q)
+#pragma unroll
+              for (int b = 0; b < NB; ++b) acc[q][b] += dot_hidden<T>(wv[q][u], hs + (size_t)b * r, r, c);
+          }
+        }
       }
 #pragma unroll
       for (int q = 0; q < R; ++q) {
@@ -280,12 +298,10 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   for (int i = threadIdx.x; i < nwl; i += kThreads)
     if (smask[i]) atomicOr(&mask_words[wfirst + i], smask[i]);
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&hdr->done, 1u) == gridDim.x - 1);
+  if (threadIdx.x == 0) s_last = (ticket_acq_rel(&hdr->done) == gridDim.x - 1);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   // ---- compaction by the last CTA: block-wide exclusive scan of popcounts ----
   const int wpt = (n_words + kThreads - 1) / kThreads;
   const int wbeg = min(n_words, threadIdx.x * wpt);
@@ -312,6 +328,272 @@ __global__ void __launch_bounds__(kThreads)
     }
   }
   if (threadIdx.x == kThreads - 1) {
+    *count = off;
+    hdr->done = 0u;
+  }
+}
+
+// ======================================================================== //
+// predictor GEMVs fed by a bulk-copy ring                                  //
+// ======================================================================== //
+
+// Shared-memory layout of the ring GEMVs: NSL slots of CR rows of K elements,
+// plus the staged activation vector(s).
+struct RingLayout {
+  size_t full, empty, vec, ring, total;
+};
+__host__ __device__ inline RingLayout ring_layout(int NSL, int CR, int K, int esz, size_t vec_bytes) {
+  RingLayout L;
+  size_t o = 0;
+  L.full = o;  o += (size_t)NSL * 8;
+  L.empty = o; o += (size_t)NSL * 8;
+  o = align_up(o, 128);
+  L.vec = o;   o += vec_bytes;
+  o = align_up(o, 128);
+  L.ring = o;  o += (size_t)NSL * CR * K * esz;
+  L.total = o;
+  return L;
+}
+
+constexpr int kRingWarps = 8;   // consumer warps; warp 8 is the producer
+
+// Issue the bulk copy of chunk i of this CTA's contiguous row slice.
+template <typename T>
+__device__ __forceinline__ void ring_issue(const T *W, int K, int row0, int row1, int CR, int NSL, int i,
+                                           T *ring, uint64_t *full) {
+  const int s = i % NSL;
+  const int ra = row0 + i * CR;
+  const int rb = min(row1, ra + CR);
+  const uint32_t bytes = (uint32_t)((size_t)(rb - ra) * K * sizeof(T));
+  mbar_arrive_expect_tx(&full[s], bytes);
+  bulk_g2s(ring + (size_t)s * CR * K, W + (size_t)ra * K, bytes, &full[s]);
+}
+
+// Producer loop for chunks [first, nch): waits for slot release, then issues.
+template <typename T>
+__device__ __forceinline__ bool ring_produce(const T *W, int K, int row0, int row1, int CR, int NSL, int first,
+                                             int nch, T *ring, uint64_t *full, uint64_t *empty) {
+  for (int i = first; i < nch; ++i) {
+    const int s = i % NSL;
+    if (i >= NSL && !mbar_wait(&empty[s], (uint32_t)((i / NSL) - 1) & 1u, kWaitNs)) return false;
+    ring_issue(W, K, row0, row1, CR, NSL, i, ring, full);
+  }
+  return true;
+}
+
+// Layer 1 of the predictor, B <= NB tokens: h = max(W1 x + b1, 0).  CTA c's
+// rows [c*rpc, (c+1)*rpc) are contiguous in memory; the producer warp copies
+// them in chunks of CR rows into an NSL-slot ring, the first chunks before the
+// kernel waits on its predecessor (weights do not depend on it).  It also
+// L2-prefetches this CTA's share of W2 for the second layer.
+template <typename T, int NB>
+__global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
+    k_pred1_ring(const T *__restrict__ W1, const float *__restrict__ b1, const T *__restrict__ x, int d, int r,
+                 int B, int rpc, int CR, int NSL, float *__restrict__ h, uint32_t *__restrict__ mask_words,
+                 int n_words, const T *__restrict__ W2, int n, int32_t *__restrict__ err, int prefetch) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int V = Vec<T>::N;
+  const RingLayout L = ring_layout(NSL, CR, d, (int)sizeof(T), (size_t)NB * d * sizeof(T));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + L.empty);
+  T *xs = reinterpret_cast<T *>(smem + L.vec);
+  T *ring = reinterpret_cast<T *>(smem + L.ring);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * rpc, row1 = min(r, row0 + rpc);
+  const int nch = row0 < row1 ? (row1 - row0 + CR - 1) / CR : 0;
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < NSL; ++q) {
+      mbar_init(&full[q], 1);
+      mbar_init(&empty[q], kRingWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == kRingWarps && lane == 0) {
+    for (int i = 0; i < min(nch, NSL); ++i) ring_issue(W1, d, row0, row1, CR, NSL, i, ring, full);
+  }
+  if (prefetch && warp == kRingWarps) {
+    const int w0 = (int)(((long long)n * blockIdx.x) / gridDim.x);
+    const int w1 = (int)(((long long)n * (blockIdx.x + 1)) / gridDim.x);
+    if (w0 < w1) {
+      const size_t bytes = (size_t)(w1 - w0) * r * sizeof(T);
+      const unsigned char *base = reinterpret_cast<const unsigned char *>(W2 + (size_t)w0 * r);
+      for (size_t o = (size_t)lane * 16384; o < bytes; o += 32 * 16384)
+        prefetch_l2(base + o, (uint32_t)min((size_t)16384, bytes - o));
+    }
+  }
+  // the next kernel reads only weights before it waits on this one
+  pdl_trigger();
+  pdl_wait();
+  for (int w = blockIdx.x * blockDim.x + threadIdx.x; w < n_words; w += gridDim.x * blockDim.x) mask_words[w] = 0u;
+  if (warp == kRingWarps) {
+    if (lane == 0 && !ring_produce(W1, d, row0, row1, CR, NSL, NSL, nch, ring, full, empty))
+      flag_error(err, kErrTimeout);
+  } else {
+    const int nvec = d / V;
+    for (int i = threadIdx.x; i < NB * nvec; i += kRingWarps * kWarp) {
+      const int b = i / nvec, c = i - b * nvec;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (b < B) v = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)b * d + (size_t)c * V));
+      *reinterpret_cast<uint4 *>(xs + (size_t)b * d + (size_t)c * V) = v;
+    }
+    named_sync(1, kRingWarps * kWarp);
+    bool ok = true;
+    for (int i = 0; i < nch; ++i) {
+      const int sl = i % NSL;
+      if (ok && !mbar_wait(&full[sl], (uint32_t)(i / NSL) & 1u, kWaitNs)) {
+        if (lane == 0) flag_error(err, kErrTimeout);
+        ok = false;
+      }
+      const int ra = row0 + i * CR, rb = min(row1, ra + CR);
+      for (int row = ra + warp; row < rb && ok; row += kRingWarps) {
+        const T *wr = ring + ((size_t)sl * CR + (row - ra)) * d;
+        float acc[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+        for (int c = lane; c < nvec; c += kWarp) {
+          const uint4 wv = *reinterpret_cast<const uint4 *>(wr + (size_t)c * V);
+#pragma unroll
+          for (int b = 0; b < NB; ++b)
+            acc[b] = Vec<T>::dot(wv, *reinterpret_cast<const uint4 *>(xs + (size_t)b * d + (size_t)c * V), acc[b]);
+        }
+        const float bias = __ldg(b1 + row);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const float sum = warp_sum(acc[b]);
+          if (lane == b && b < B) h[(size_t)b * r + row] = fmaxf(sum + bias, 0.f);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[sl]);
+    }
+  }
+}
+
+// Layer 2 + threshold + union + compaction, B <= NB tokens, with W2 rows fed
+// by the bulk-copy ring (first chunks issued before the wait).  Bits, ticket
+// and the last-CTA compaction are as in k_pred_l2.
+template <typename T, int NB>
+__global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
+    k_pred2_ring(const T *__restrict__ W2, const float *__restrict__ b2, const float *__restrict__ h, int r, int n,
+                 int B, float thr, int rpc, int CR, int NSL, uint32_t *__restrict__ mask_words, int n_words,
+                 int32_t *__restrict__ idx, int32_t *__restrict__ count, Header *__restrict__ hdr) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int V = Vec<T>::N;
+  constexpr int NT = (kRingWarps + 1) * kWarp;
+  const int nwl_max = rpc / 32 + 2;
+  const RingLayout L = ring_layout(NSL, CR, r, (int)sizeof(T), (size_t)NB * r * 4 + (size_t)nwl_max * 4);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + L.empty);
+  float *hs = reinterpret_cast<float *>(smem + L.vec);
+  uint32_t *smask = reinterpret_cast<uint32_t *>(smem + L.vec + (size_t)NB * r * 4);
+  T *ring = reinterpret_cast<T *>(smem + L.ring);
+  __shared__ int s_last;
+  __shared__ int s_wsum[NT / kWarp];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * rpc, row1 = min(n, row0 + rpc);
+  const int nch = row0 < row1 ? (row1 - row0 + CR - 1) / CR : 0;
+  const int wfirst = row0 >> 5;
+  const int nwl = (row0 < row1) ? (((row1 - 1) >> 5) - wfirst + 1) : 0;
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < NSL; ++q) {
+      mbar_init(&full[q], 1);
+      mbar_init(&empty[q], kRingWarps);
+    }
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < nwl; i += NT) smask[i] = 0u;
+  __syncthreads();
+  if (warp == kRingWarps && lane == 0) {
+    for (int i = 0; i < min(nch, NSL); ++i) ring_issue(W2, r, row0, row1, CR, NSL, i, ring, full);
+  }
+  pdl_trigger();
+  pdl_wait();
+  if (warp == kRingWarps) {
+    if (lane == 0 && !ring_produce(W2, r, row0, row1, CR, NSL, NSL, nch, ring, full, empty))
+      flag_error(&hdr->err, kErrTimeout);
+  } else {
+    for (int i = threadIdx.x; i < NB * r; i += kRingWarps * kWarp) {
+      const int b = i / r, e = i - b * r;
+      const float v = (b < B) ? __ldcg(h + (size_t)b * r + e) : 0.f;
+      int pos = e;
+      if (sizeof(T) == 2) {
+        const int c = e >> 3, q = e & 7;
+        pos = (q < 4) ? (c * 4 + q) : (r / 2 + c * 4 + (q - 4));
+      }
+      hs[(size_t)b * r + pos] = v;
+    }
+    named_sync(1, kRingWarps * kWarp);
+    const int nvec = r / V;
+    bool ok = true;
+    for (int i = 0; i < nch; ++i) {
+      const int sl = i % NSL;
+      if (ok && !mbar_wait(&full[sl], (uint32_t)(i / NSL) & 1u, kWaitNs)) {
+        if (lane == 0) flag_error(&hdr->err, kErrTimeout);
+        ok = false;
+      }
+      const int ra = row0 + i * CR, rb = min(row1, ra + CR);
+      for (int row = ra + warp; row < rb && ok; row += kRingWarps) {
+        const T *wr = ring + ((size_t)sl * CR + (row - ra)) * r;
+        float acc[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+        for (int c = lane; c < nvec; c += kWarp) {
+          const uint4 wv = *reinterpret_cast<const uint4 *>(wr + (size_t)c * V);
+#pragma unroll
+          for (int b = 0; b < NB; ++b) acc[b] += dot_hidden<T>(wv, hs + (size_t)b * r, r, c);
+        }
+        bool on = false;
+        const float bias = __ldg(b2 + row);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const float z = warp_sum(acc[b]) + bias;
+          on |= (b < B) && (z > thr);
+        }
+        if (lane == 0 && on) atomicOr(&smask[(row >> 5) - wfirst], 1u << (row & 31));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[sl]);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nwl; i += NT)
+    if (smask[i]) atomicOr(&mask_words[wfirst + i], smask[i]);
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (ticket_acq_rel(&hdr->done) == gridDim.x - 1);
+  __syncthreads();
+  if (!s_last) return;
+  // ---- compaction by the last CTA: block-wide exclusive scan of popcounts ----
+  const int wpt = (n_words + NT - 1) / NT;
+  const int wbeg = min(n_words, (int)threadIdx.x * wpt);
+  const int wend = min(n_words, wbeg + wpt);
+  uint32_t wv[8];
+  int local = 0;
+  for (int w = wbeg, q = 0; w < wend; ++w, ++q) {
+    const uint32_t m = ld_cg_u32(mask_words + w);
+    if (q < 8) wv[q] = m;
+    local += __popc(m);
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < kWarp; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == kWarp - 1) s_wsum[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += s_wsum[w];
+  int off = before + incl - local;
+  for (int w = wbeg, q = 0; w < wend; ++w, ++q) {
+    uint32_t m = q < 8 ? wv[q] : ld_cg_u32(mask_words + w);
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      idx[off++] = w * 32 + bit;
+      m &= m - 1u;
+    }
+  }
+  if (threadIdx.x == NT - 1) {
     *count = off;
     hdr->done = 0u;
   }
@@ -474,20 +756,333 @@ __global__ void __launch_bounds__(kThreads)
     }
   }
   if (S == 1) return;
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&hdr->tile_done[tile], 1u) == (unsigned)S - 1u);
+  if (threadIdx.x == 0) s_last = (ticket_acq_rel(&hdr->tile_done[tile]) == (unsigned)S - 1u);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   const int tw = min(TW, d - col0);
   for (int i = threadIdx.x; i < B * tw; i += kThreads) {
     const int b = i / tw, c = i - b * tw;
     float s = 0.f;
-    for (int q = 0; q < S; ++q) s += ld_cg_f32(part + ((size_t)q * B + b) * d + col0 + c);
+    for (int q0 = 0; q0 < S; q0 += 16) {   // 16 loads in flight, summed in split order
+      float v[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        v[q] = q0 + q < S ? ld_cg_f32(part + ((size_t)(q0 + q) * B + b) * d + col0 + c) : 0.f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (q0 + q < S) s += v[q];
+    }
     y[(size_t)b * d + col0 + c] = s;
   }
   if (threadIdx.x == 0) hdr->tile_done[tile] = 0u;
+}
+
+// ======================================================================== //
+// fused sparse FFN: bulk-copy ring + cluster reduction                     //
+// ======================================================================== //
+
+// Shared-memory layout of k_sparse_ffn for NS ring slots of M rows of d elements.
+struct FusedLayout {
+  int NS, grp;
+  size_t full, empty, kslot, pd, x, stage, red, total;
+};
+
+__host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int esz, int NB) {
+  FusedLayout L;
+  L.NS = NS;
+  L.grp = NS / 2 > 0 ? NS / 2 : 1;
+  size_t o = 0;
+  L.full = o;  o += (size_t)NS * 8;
+  L.empty = o; o += (size_t)NS * 8;
+  L.kslot = o; o += (size_t)NS * 4;
+  o = align_up(o, 16);
+  L.pd = o;    o += (size_t)kFusedWarps * L.grp * 2 * NB * 4;
+  o = align_up(o, 128);
+  L.x = o;     o += (size_t)NB * d * esz;
+  o = align_up(o, 128);
+  L.stage = o; o += (size_t)NS * M * d * esz;
+  const size_t red = (size_t)NB * d * 4;
+  if (red <= (size_t)NS * M * d * esz) {
+    L.red = L.stage;
+  } else {
+    o = align_up(o, 128);
+    L.red = o;
+    o += red;
+  }
+  L.total = o;
+  return L;
+}
+
+// One kernel for the whole neuron-sparse FFN of B <= NB tokens.
+//
+// CTA c of a grid of G takes list positions [c*cnt/G, (c+1)*cnt/G).  Warp
+// kFusedWarps is the producer: one lane streams, for each of its neurons k,
+// the rows Wg[k], Wu[k], WdT[k] into a ring of NS shared-memory slots with
+// cp.async.bulk, completing on the slot's "full" mbarrier.  The 8 consumer
+// warps split d: each owns chunks (q*8 + warp)*32 + lane, so every warp reads
+// every slot.  Neurons are consumed in groups of NS/2 (the other half of the
+// ring is being refilled): partial gate/up dots over the warp's d-slice go to
+// shared memory, one named barrier, every warp sums the 8 partials in warp
+// order, applies ReLU(g + b) * u (or ReLU(u + b)), and accumulates
+// a * WdT[k] into its registers; then it releases the slot ("empty").
+// At the end the CTA's y partial is reduced across the cluster through DSMEM
+// (CTA rank q sums column block q in rank order) and across clusters by the
+// last cluster to finish each block (atomic ticket), in cluster order.
+template <typename T, int NB, int MAXQ, bool REGLU>
+__global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
+    k_sparse_ffn(const T *__restrict__ Wg, const T *__restrict__ Wu, const T *__restrict__ WdT,
+                 const float *__restrict__ bias, const T *__restrict__ x, int d, int n, int B,
+                 const int32_t *__restrict__ idx, const int32_t *__restrict__ count, int NS,
+                 float *__restrict__ part, float *__restrict__ y, Header *__restrict__ hdr) {
+  namespace cg = cooperative_groups;
+  constexpr int V = Vec<T>::N;
+  constexpr int M = REGLU ? 3 : 2;
+  constexpr int NW = kFusedWarps;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_last;
+  __shared__ int s_fail;
+  const FusedLayout L = fused_layout(NS, d, M, (int)sizeof(T), NB);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + L.empty);
+  int *kslot = reinterpret_cast<int *>(smem + L.kslot);
+  float *pd = reinterpret_cast<float *>(smem + L.pd);
+  T *xs = reinterpret_cast<T *>(smem + L.x);
+  T *stage = reinterpret_cast<T *>(smem + L.stage);
+  float *red = reinterpret_cast<float *>(smem + L.red);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nvec = d / V;
+  const int grp = L.grp;
+  int32_t *err = &hdr->err;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NW);
+      kslot[s] = -1;
+    }
+    fence_mbar_init();
+    s_fail = 0;
+  }
+  __syncthreads();
+  // The next kernel only prefetches weights before it waits on this one.
+  pdl_trigger();
+  pdl_wait();
+
+  int cnt = n;
+  if (idx) {
+    const int c = ld_cg_i32(count);
+    if (c < 0 || c > n) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(err, kErrIndex);
+    }
+    cnt = max(0, min(c, n));
+  }
+  const int G = gridDim.x;
+  const int js = (int)(((long long)cnt * blockIdx.x) / G);
+  const int je = (int)(((long long)cnt * (blockIdx.x + 1)) / G);
+  const int nl = je - js;
+
+  float acc[MAXQ][V][NB];
+#pragma unroll
+  for (int q = 0; q < MAXQ; ++q)
+#pragma unroll
+    for (int e = 0; e < V; ++e)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) acc[q][e][b] = 0.f;
+
+  if (warp == NW) {
+    // ------------------------------------------------------------ producer --
+    // The whole warp walks the list; indices are fetched 32 at a time with one
+    // coalesced load and broadcast by shuffle; lane 0 issues the copies.
+    const uint32_t row_bytes = (uint32_t)((size_t)d * sizeof(T));
+    int kreg = 0;
+    bool stop = false;
+    for (int i = 0; i < nl && !stop; ++i) {
+      if ((i & 31) == 0) {
+        const int j = js + i + lane;
+        kreg = (j < je) ? (idx ? ld_cg_i32(idx + j) : j) : -1;
+      }
+      const int k = __shfl_sync(0xffffffffu, kreg, i & 31);
+      if (lane == 0) {
+        const int s = i % NS;
+        if (i >= NS && !mbar_wait(&empty[s], (uint32_t)((i / NS) - 1) & 1u, kWaitNs)) {
+          flag_error(err, kErrTimeout);
+          s_fail = 1;
+          stop = true;
+        } else if ((unsigned)k >= (unsigned)n) {
+          flag_error(err, kErrIndex);
+          kslot[s] = -1;
+          mbar_arrive(&full[s]);
+        } else {
+          kslot[s] = k;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)M * row_bytes);
+          T *dst = stage + (size_t)s * M * d;
+          if constexpr (REGLU) {
+            bulk_g2s(dst, Wg + (size_t)k * d, row_bytes, &full[s]);
+            bulk_g2s(dst + d, Wu + (size_t)k * d, row_bytes, &full[s]);
+            bulk_g2s(dst + 2 * (size_t)d, WdT + (size_t)k * d, row_bytes, &full[s]);
+          } else {
+            bulk_g2s(dst, Wu + (size_t)k * d, row_bytes, &full[s]);
+            bulk_g2s(dst + d, WdT + (size_t)k * d, row_bytes, &full[s]);
+          }
+        }
+      }
+      stop = __shfl_sync(0xffffffffu, stop, 0);
+    }
+  } else {
+    // ----------------------------------------------------------- consumers --
+    for (int i = threadIdx.x; i < NB * nvec; i += NW * kWarp) {
+      const int b = i / nvec, c = i - b * nvec;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (b < B) v = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)b * d + (size_t)c * V));
+      *reinterpret_cast<uint4 *>(xs + (size_t)b * d + (size_t)c * V) = v;
+    }
+    named_sync(1, NW * kWarp);
+    bool ok = true;
+    for (int g0 = 0; g0 < nl; g0 += grp) {
+      const int gn = min(grp, nl - g0);
+      for (int q = 0; q < gn; ++q) {
+        const int i = g0 + q, s = i % NS;
+        if (ok && !mbar_wait(&full[s], (uint32_t)(i / NS) & 1u, kWaitNs)) {
+          if (lane == 0) flag_error(err, kErrTimeout);
+          ok = false;
+        }
+        float pg[NB], pu[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) pg[b] = pu[b] = 0.f;
+        if (ok && kslot[s] >= 0) {
+          const T *ru = stage + (size_t)s * M * d + (REGLU ? d : 0);
+          const T *rg = stage + (size_t)s * M * d;
+#pragma unroll
+          for (int qq = 0; qq < MAXQ; ++qq) {
+            const int ch = (qq * NW + warp) * kWarp + lane;
+            if (ch < nvec) {
+              const uint4 wu = *reinterpret_cast<const uint4 *>(ru + (size_t)ch * V);
+              uint4 wg = wu;
+              if constexpr (REGLU) wg = *reinterpret_cast<const uint4 *>(rg + (size_t)ch * V);
+#pragma unroll
+              for (int b = 0; b < NB; ++b) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)b * d + (size_t)ch * V);
+                pu[b] = Vec<T>::dot(wu, xv, pu[b]);
+                if constexpr (REGLU) pg[b] = Vec<T>::dot(wg, xv, pg[b]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          pu[b] = warp_sum(pu[b]);
+          if constexpr (REGLU) pg[b] = warp_sum(pg[b]);
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            pd[(((size_t)warp * grp + q) * 2 + 0) * NB + b] = pg[b];
+            pd[(((size_t)warp * grp + q) * 2 + 1) * NB + b] = pu[b];
+          }
+        }
+      }
+      named_sync(1, NW * kWarp);
+      for (int q = 0; q < gn; ++q) {
+        const int i = g0 + q, s = i % NS;
+        const int k = kslot[s];
+        float a[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          float g = 0.f, u = 0.f;
+#pragma unroll
+          for (int w = 0; w < NW; ++w) {
+            g += pd[(((size_t)w * grp + q) * 2 + 0) * NB + b];
+            u += pd[(((size_t)w * grp + q) * 2 + 1) * NB + b];
+          }
+          float v = 0.f;
+          if (k >= 0 && b < B) {
+            const float bk = __ldg(bias + k);
+            v = REGLU ? fmaxf(g + bk, 0.f) * u : fmaxf(u + bk, 0.f);
+          }
+          a[b] = v;
+        }
+        if (ok && k >= 0) {
+          const T *rd = stage + (size_t)s * M * d + (size_t)(M - 1) * d;
+#pragma unroll
+          for (int qq = 0; qq < MAXQ; ++qq) {
+            const int ch = (qq * NW + warp) * kWarp + lane;
+            if (ch < nvec) {
+              float f[V];
+              Vec<T>::to_float(*reinterpret_cast<const uint4 *>(rd + (size_t)ch * V), f);
+#pragma unroll
+              for (int e = 0; e < V; ++e)
+#pragma unroll
+                for (int b = 0; b < NB; ++b) acc[qq][e][b] = fmaf(a[b], f[e], acc[qq][e][b]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      named_sync(1, NW * kWarp);
+    }
+    if (!ok) s_fail = 1;
+  }
+  __syncthreads();
+  // -------------------------------------------------------- reductions --
+  if (warp < NW) {
+#pragma unroll
+    for (int qq = 0; qq < MAXQ; ++qq) {
+      const int ch = (qq * NW + warp) * kWarp + lane;
+      if (ch < nvec) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int e = 0; e < V; ++e) red[(size_t)b * d + (size_t)ch * V + e] = acc[qq][e][b];
+      }
+    }
+  }
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();
+  const int crank = (int)cluster.block_rank();
+  const int ncl = G / kCluster;
+  const int cid = blockIdx.x / kCluster;
+  const int blk = ((nvec + kCluster - 1) / kCluster) * V;   // columns per block
+  const int c0 = min(d, crank * blk), c1 = min(d, c0 + blk);
+  const int w = c1 - c0;
+  const float *peer[kCluster];
+#pragma unroll
+  for (int r = 0; r < kCluster; ++r) peer[r] = cluster.map_shared_rank(red, r);
+  for (int i = threadIdx.x; i < B * w; i += blockDim.x) {
+    const int b = i / w, col = c0 + (i - b * w);
+    float v[kCluster];
+#pragma unroll
+    for (int r = 0; r < kCluster; ++r) v[r] = peer[r][(size_t)b * d + col];
+    float sum = 0.f;
+#pragma unroll
+    for (int r = 0; r < kCluster; ++r) sum += v[r];
+    if (ncl == 1)
+      y[(size_t)b * d + col] = sum;
+    else
+      part[((size_t)cid * B + b) * d + col] = sum;
+  }
+  cluster.sync();
+  if (ncl == 1) return;
+  if (threadIdx.x == 0) s_last = (ticket_acq_rel(&hdr->tile_done[crank]) == (unsigned)ncl - 1u);
+  __syncthreads();
+  if (!s_last) return;
+  // all partials of an output are loaded before any is added (one L2 round
+  // trip, not one per cluster); the sum runs in cluster order
+  for (int i = threadIdx.x; i < B * w; i += blockDim.x) {
+    const int b = i / w, col = c0 + (i - b * w);
+    float sum = 0.f;
+    for (int q0 = 0; q0 < ncl; q0 += 4) {
+      float v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[q] = q0 + q < ncl ? ld_cg_f32(part + ((size_t)(q0 + q) * B + b) * d + col) : 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q0 + q < ncl) sum += v[q];
+    }
+    y[(size_t)b * d + col] = sum;
+  }
+  if (threadIdx.x == 0) hdr->tile_done[crank] = 0u;
 }
 
 // ======================================================================== //
@@ -589,6 +1184,14 @@ bool pdl_enabled() {
   static int on = env_flag("ASFFN_PDL", 1);
   return on != 0;
 }
+size_t fused_smem_budget() {
+  static size_t kb = (size_t)env_flag("ASFFN_FUSED_SMEM_KB", (int)(kFusedSmemDefault / 1024));
+  return std::min<size_t>(std::max<size_t>(kb, 32), 220) * 1024;
+}
+bool fused_enabled() {
+  static int on = env_flag("ASFFN_FUSED", 1);
+  return on != 0;
+}
 int prefetch_enabled() {
   static int on = env_flag("ASFFN_PREFETCH", 1);
   return on;
@@ -616,6 +1219,70 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// Launch with a thread-block cluster of `cl` CTAs along x (plus PDL).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, int cl, cudaStream_t st,
+                           Args... args) {
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute((const void *)kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cl;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// Clusters of `cl` CTAs that can be resident at once (cached per kernel/device).
+template <typename... KArgs>
+int max_clusters(void (*kern)(KArgs...), int threads, size_t smem, int cl) {
+  static std::mutex mu;
+  static std::map<std::pair<const void *, std::pair<int, size_t>>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto key = std::make_pair((const void *)kern, std::make_pair(dev, smem));
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute((const void *)kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(cl * 32);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (const void *)kern, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 0;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  cache[key] = n;
+  return n;
+}
+
 inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 inline size_t r256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -635,7 +1302,9 @@ size_t pred_scratch(const asf_predictor *p, int B) {
   return r256((size_t)n_words_of(p->n) * 4) + r256((size_t)B * p->r * 4);
 }
 size_t ffn_scratch(const asf_ffn *f, int B) {
-  return r256((size_t)f->n * B * 4) + r256((size_t)down_splits(f) * B * f->d * 4);
+  const size_t two_kernel = r256((size_t)f->n * B * 4) + r256((size_t)down_splits(f) * B * f->d * 4);
+  const size_t fused = r256((size_t)kMaxClusters * B * f->d * 4);
+  return std::max(two_kernel, fused);
 }
 
 asf_status check_pred(const asf_predictor *p) {
@@ -685,8 +1354,9 @@ cudaError_t run_pred_l1(const asf_predictor *p, const void *x, int B, float *h, 
   const int rpc = (p->r + sms - 1) / sms;
   const int grid = (p->r + rpc - 1) / rpc;
   const size_t smem = (size_t)NB * p->d * sizeof(T);
-  return launch(k_pred_l1<T, NB, 8>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W1, p->b1,
-                (const T *)x, p->d, p->r, B, rpc, h, mask, n_words_of(p->n), prefetch_enabled());
+  return launch(k_pred_l1<T, NB, (NB <= 2 ? 16 : 8)>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W1, p->b1,
+                (const T *)x, p->d, p->r, B, rpc, h, mask, n_words_of(p->n), (const T *)p->W2, p->n,
+                prefetch_enabled());
 }
 
 template <typename T, int NB>
@@ -696,10 +1366,107 @@ cudaError_t run_pred_l2(const asf_predictor *p, int B, float thr, const float *h
   const int rpc = (p->n + sms - 1) / sms;
   const int grid = (p->n + rpc - 1) / rpc;
   const size_t smem = (size_t)NB * p->r * 4 + ((size_t)rpc / 32 + 2) * 4;
-  return launch(k_pred_l2<T, NB, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W2, p->b2, h, p->r,
+  return launch(k_pred_l2<T, NB, (NB <= 2 ? 4 : 2), (NB <= 2 ? 4 : 2)>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W2, p->b2, h, p->r,
                 p->n, B, thr, rpc, mask, n_words_of(p->n), idx, count, hdr, prefetch_enabled());
 }
 
+constexpr size_t kRingChunk = 32 * 1024;    // bytes per bulk copy of a ring slot
+constexpr size_t kRing1Smem = 80 * 1024;     // layer-1 ring + x: fits beside the fused FFN
+constexpr size_t kRing2Smem = 140 * 1024;
+
+// rows per chunk and slots for a ring over rows of row_bytes within budget
+bool ring_shape(size_t row_bytes, size_t vec_bytes, size_t budget, int rpc, int &CR, int &NSL) {
+  CR = (int)std::max<size_t>(1, kRingChunk / row_bytes);
+  CR = std::min(CR, std::max(1, rpc));
+  for (NSL = 4; NSL >= 2; --NSL)
+    if (ring_layout(NSL, CR, 1, (int)row_bytes, vec_bytes).total <= budget) return true;
+  return false;
+}
+
+template <typename T, int NB>
+cudaError_t run_pred1_ring(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, int32_t *err,
+                           cudaStream_t st, bool &used) {
+  const int sms = sm_count();
+  const int rpc = (p->r + sms - 1) / sms;
+  const int grid = (p->r + rpc - 1) / rpc;
+  int CR, NSL;
+  used = ring_shape((size_t)p->d * sizeof(T), (size_t)NB * p->d * sizeof(T), kRing1Smem, rpc, CR, NSL);
+  if (!used) return cudaSuccess;
+  const size_t smem = ring_layout(NSL, CR, p->d, (int)sizeof(T), (size_t)NB * p->d * sizeof(T)).total;
+  return launch(k_pred1_ring<T, NB>, dim3(grid), dim3((kRingWarps + 1) * kWarp), smem, st, (const T *)p->W1,
+                p->b1, (const T *)x, p->d, p->r, B, rpc, CR, NSL, h, mask, n_words_of(p->n), (const T *)p->W2,
+                p->n, err, prefetch_enabled());
+}
+
+template <typename T, int NB>
+cudaError_t run_pred2_ring(const asf_predictor *p, int B, float thr, const float *h, uint32_t *mask, int32_t *idx,
+                           int32_t *count, Header *hdr, cudaStream_t st, bool &used) {
+  const int sms = sm_count();
+  const int rpc = (p->n + sms - 1) / sms;
+  const int grid = (p->n + rpc - 1) / rpc;
+  const size_t vec = (size_t)NB * p->r * 4 + ((size_t)rpc / 32 + 2) * 4;
+  int CR, NSL;
+  used = ring_shape((size_t)p->r * sizeof(T), vec, kRing2Smem, rpc, CR, NSL);
+  if (!used) return cudaSuccess;
+  const size_t smem = ring_layout(NSL, CR, p->r, (int)sizeof(T), vec).total;
+  return launch(k_pred2_ring<T, NB>, dim3(grid), dim3((kRingWarps + 1) * kWarp), smem, st, (const T *)p->W2,
+                p->b2, h, p->r, p->n, B, thr, rpc, CR, NSL, mask, n_words_of(p->n), idx, count, hdr);
+}
+
+bool ring_enabled() {
+  static int on = env_flag("ASFFN_RING", 1);
+  return on != 0;
+}
+
+// largest token group in {1, 2, 4, 8} covering B (B <= 8)
+inline int nb_cover(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 8; }
+
+template <typename T>
+cudaError_t pred1_ring_any(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, int32_t *err,
+                           cudaStream_t st, bool &used) {
+  switch (nb_cover(B)) {
+    case 1: return run_pred1_ring<T, 1>(p, x, B, h, mask, err, st, used);
+    case 2: return run_pred1_ring<T, 2>(p, x, B, h, mask, err, st, used);
+    case 4: return run_pred1_ring<T, 4>(p, x, B, h, mask, err, st, used);
+    default: return run_pred1_ring<T, 8>(p, x, B, h, mask, err, st, used);
+  }
+}
+
+template <typename T>
+cudaError_t pred2_ring_any(const asf_predictor *p, int B, float thr, const float *h, uint32_t *mask, int32_t *idx,
+                           int32_t *count, Header *hdr, cudaStream_t st, bool &used) {
+  switch (nb_cover(B)) {
+    case 1: return run_pred2_ring<T, 1>(p, B, thr, h, mask, idx, count, hdr, st, used);
+    case 2: return run_pred2_ring<T, 2>(p, B, thr, h, mask, idx, count, hdr, st, used);
+    case 4: return run_pred2_ring<T, 4>(p, B, thr, h, mask, idx, count, hdr, st, used);
+    default: return run_pred2_ring<T, 8>(p, B, thr, h, mask, idx, count, hdr, st, used);
+  }
+}
+
+template <typename T>
+cudaError_t pred1_reg_any(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, cudaStream_t st) {
+  switch (pick_nb(B, (size_t)p->d * sizeof(T))) {
+    case 1: return run_pred_l1<T, 1>(p, x, B, h, mask, st);
+    case 2: return run_pred_l1<T, 2>(p, x, B, h, mask, st);
+    case 4: return run_pred_l1<T, 4>(p, x, B, h, mask, st);
+    default: return run_pred_l1<T, 8>(p, x, B, h, mask, st);
+  }
+}
+
+template <typename T>
+cudaError_t pred2_reg_any(const asf_predictor *p, int B, float thr, const float *h, uint32_t *mask, int32_t *idx,
+                          int32_t *count, Header *hdr, cudaStream_t st) {
+  switch (pick_nb(B, (size_t)p->r * 4)) {
+    case 1: return run_pred_l2<T, 1>(p, B, thr, h, mask, idx, count, hdr, st);
+    case 2: return run_pred_l2<T, 2>(p, B, thr, h, mask, idx, count, hdr, st);
+    case 4: return run_pred_l2<T, 4>(p, B, thr, h, mask, idx, count, hdr, st);
+    default: return run_pred_l2<T, 8>(p, B, thr, h, mask, idx, count, hdr, st);
+  }
+}
+
+// Layer 1 then layer 2 + compaction.  Batches of up to 8 tokens use the
+// bulk-copy ring kernels when their slices fit; larger batches use the
+// register-streaming kernels, which loop over token groups.
 template <typename T>
 asf_status predict_t(const asf_predictor *p, const void *x, int B, float thr, int32_t *idx, int32_t *count,
                      void *ws, cudaStream_t st) {
@@ -707,22 +1474,15 @@ asf_status predict_t(const asf_predictor *p, const void *x, int B, float thr, in
   Header *hdr = reinterpret_cast<Header *>(base);
   uint32_t *mask = reinterpret_cast<uint32_t *>(base + kHeaderBytes);
   float *h = reinterpret_cast<float *>(base + kHeaderBytes + r256((size_t)n_words_of(p->n) * 4));
-  const int nb1 = pick_nb(B, (size_t)p->d * sizeof(T));
-  const int nb2 = pick_nb(B, (size_t)p->r * 4);
-  cudaError_t e;
-  switch (nb1) {
-    case 1: e = run_pred_l1<T, 1>(p, x, B, h, mask, st); break;
-    case 2: e = run_pred_l1<T, 2>(p, x, B, h, mask, st); break;
-    case 4: e = run_pred_l1<T, 4>(p, x, B, h, mask, st); break;
-    default: e = run_pred_l1<T, 8>(p, x, B, h, mask, st); break;
-  }
+  const bool ring = B <= 8 && ring_enabled();
+  bool used = false;
+  cudaError_t e = cudaSuccess;
+  if (ring) e = pred1_ring_any<T>(p, x, B, h, mask, &hdr->err, st, used);
+  if (e == cudaSuccess && !used) e = pred1_reg_any<T>(p, x, B, h, mask, st);
   if (e != cudaSuccess) return ASF_ERR_CUDA;
-  switch (nb2) {
-    case 1: e = run_pred_l2<T, 1>(p, B, thr, h, mask, idx, count, hdr, st); break;
-    case 2: e = run_pred_l2<T, 2>(p, B, thr, h, mask, idx, count, hdr, st); break;
-    case 4: e = run_pred_l2<T, 4>(p, B, thr, h, mask, idx, count, hdr, st); break;
-    default: e = run_pred_l2<T, 8>(p, B, thr, h, mask, idx, count, hdr, st); break;
-  }
+  used = false;
+  if (ring) e = pred2_ring_any<T>(p, B, thr, h, mask, idx, count, hdr, st, used);
+  if (e == cudaSuccess && !used) e = pred2_reg_any<T>(p, B, thr, h, mask, idx, count, hdr, st);
   return cuda_status(e);
 }
 
@@ -733,9 +1493,9 @@ cudaError_t run_gu(const asf_ffn *f, const void *x, int B, const int32_t *idx, c
   const int grid = 2 * sm_count();
   const size_t smem = (size_t)NB * f->d * sizeof(T);
   if (f->act == ASF_ACT_REGLU)
-    return launch(k_ffn_gu<T, NB, 4, true>, dim3(grid), dim3(kThreads), smem, st, (const T *)f->Wg,
+    return launch(k_ffn_gu<T, NB, (NB <= 2 ? 8 : 4), true>, dim3(grid), dim3(kThreads), smem, st, (const T *)f->Wg,
                   (const T *)f->Wu, f->bias, (const T *)x, f->d, f->n, B, idx, count, a, err);
-  return launch(k_ffn_gu<T, NB, 4, false>, dim3(grid), dim3(kThreads), smem, st, (const T *)f->Wg,
+  return launch(k_ffn_gu<T, NB, (NB <= 2 ? 8 : 4), false>, dim3(grid), dim3(kThreads), smem, st, (const T *)f->Wg,
                 (const T *)f->Wu, f->bias, (const T *)x, f->d, f->n, B, idx, count, a, err);
 }
 
@@ -750,6 +1510,77 @@ cudaError_t run_down(const asf_ffn *f, int B, const int32_t *idx, const int32_t 
                 f->d, f->n, B, S, part, y, hdr, prefetch_enabled());
 }
 
+// ------------------------------------------------------------- fused ffn --
+int fused_maxq(const asf_ffn *f) {
+  const int nvec = f->d / vec_of(f->wdtype);
+  const int q = (nvec + kFusedWarps * kWarp - 1) / (kFusedWarps * kWarp);
+  return q <= 1 ? 1 : q <= 2 ? 2 : q <= 4 ? 4 : q <= 6 ? 6 : 0;
+}
+int fused_nb(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 0; }
+
+// Ring slots that fit the shared-memory budget (0 if fewer than two).
+int fused_slots(const asf_ffn *f, int NB) {
+  const int M = f->act == ASF_ACT_REGLU ? 3 : 2;
+  for (int ns = 16; ns >= 2; --ns)
+    if (fused_layout(ns, f->d, M, esize(f->wdtype), NB).total <= fused_smem_budget()) return ns;
+  return 0;
+}
+
+bool fused_ok(const asf_ffn *f, int B) {
+  const int nb = fused_nb(B), q = fused_maxq(f);
+  if (!nb || !q) return false;
+  if (q * vec_of(f->wdtype) * nb > 64) return false;   // y accumulators per lane
+  return fused_slots(f, nb) >= 2;
+}
+
+template <typename T, int NB, int MAXQ, bool REGLU>
+cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
+                        float *y, Header *hdr, cudaStream_t st) {
+  if constexpr (MAXQ * Vec<T>::N * NB > 64) {
+    return cudaErrorInvalidConfiguration;
+  } else {
+    const int M = REGLU ? 3 : 2;
+    const int NS = fused_slots(f, NB);
+    const FusedLayout L = fused_layout(NS, f->d, M, (int)sizeof(T), NB);
+    const int threads = (kFusedWarps + 1) * kWarp;
+    auto kern = k_sparse_ffn<T, NB, MAXQ, REGLU>;
+    int ncl = max_clusters(kern, threads, L.total, kCluster);
+    ncl = std::min(ncl, std::min(kMaxClusters, (sm_count() + kCluster - 1) / kCluster));
+    if (ncl <= 0) return cudaErrorInvalidConfiguration;
+    return launch_cluster(kern, dim3(ncl * kCluster), dim3(threads), L.total, kCluster, st, (const T *)f->Wg,
+                          (const T *)f->Wu, (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count,
+                          NS, part, y, hdr);
+  }
+}
+
+template <typename T, int NB, int MAXQ>
+cudaError_t run_fused_a(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
+                        float *y, Header *hdr, cudaStream_t st) {
+  if (f->act == ASF_ACT_REGLU) return run_fused_k<T, NB, MAXQ, true>(f, x, B, idx, count, part, y, hdr, st);
+  return run_fused_k<T, NB, MAXQ, false>(f, x, B, idx, count, part, y, hdr, st);
+}
+
+template <typename T, int NB>
+cudaError_t run_fused_q(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
+                        float *y, Header *hdr, cudaStream_t st) {
+  switch (fused_maxq(f)) {
+    case 1: return run_fused_a<T, NB, 1>(f, x, B, idx, count, part, y, hdr, st);
+    case 2: return run_fused_a<T, NB, 2>(f, x, B, idx, count, part, y, hdr, st);
+    case 4: return run_fused_a<T, NB, 4>(f, x, B, idx, count, part, y, hdr, st);
+    default: return run_fused_a<T, NB, 6>(f, x, B, idx, count, part, y, hdr, st);
+  }
+}
+
+template <typename T>
+cudaError_t run_fused(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
+                      float *y, Header *hdr, cudaStream_t st) {
+  switch (fused_nb(B)) {
+    case 1: return run_fused_q<T, 1>(f, x, B, idx, count, part, y, hdr, st);
+    case 2: return run_fused_q<T, 2>(f, x, B, idx, count, part, y, hdr, st);
+    default: return run_fused_q<T, 4>(f, x, B, idx, count, part, y, hdr, st);
+  }
+}
+
 template <typename T>
 asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *y,
                  void *ws, cudaStream_t st) {
@@ -757,6 +1588,10 @@ asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, con
   Header *hdr = reinterpret_cast<Header *>(base);
   float *a = reinterpret_cast<float *>(base + kHeaderBytes);
   float *part = reinterpret_cast<float *>(base + kHeaderBytes + r256((size_t)f->n * B * 4));
+  if (fused_ok(f, B) && fused_enabled()) {
+    float *cpart = reinterpret_cast<float *>(base + kHeaderBytes);
+    return cuda_status(run_fused<T>(f, x, B, idx, count, cpart, y, hdr, st));
+  }
   const int nbg = pick_nb(B, (size_t)f->d * sizeof(T));
   cudaError_t e;
   switch (nbg) {

@@ -1,0 +1,526 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the activation-sparse FFN path on B200.
+
+A step is one decode step of B tokens through the whole layer stack: for each
+layer, the predictor (two GEMVs, threshold, compaction) and the sparse FFN
+(gate/up gather, activation, W_down^T gather-accumulate), all in libasffn's
+kernels, replayed from one CUDA graph.  Inputs are synthetic and seeded; the
+weights of the stack (9.6 GB for the Llama2-7B shape) are far larger than L2,
+so every step reads its rows from HBM.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+instead (rank 0 only; other ranks exit without work).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-FFN tokens/s per layer stack at batch 1; achieved HBM GB/s vs roofline"
+NOMINAL_HBM_GBS = 7700.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=4096)
+    p.add_argument("--warmup", type=int, default=32)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", default="llama2_7b_reglu")
+    p.add_argument("--batch", type=int, default=1)
+    p.add_argument("--mode", choices=["predict", "sparse", "dense"], default="predict")
+    p.add_argument("--no-hot-perm", action="store_true", help="keep neuron id order")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=1024)
+    p.add_argument("--profile-steps", type=int, default=256)
+    p.add_argument("--layers", type=int, default=0,
+                   help="layers in the stack (default: the config's; fewer only for profiling runs)")
+    p.add_argument("--tokens", type=int, default=0,
+                   help="distinct tokens cycled through (default: the config's token count)")
+    p.add_argument("--reference-budget", type=float, default=90.0,
+                   help="seconds of CPU time the reference arm may spend")
+    return p.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- #
+# helpers                                                                       #
+# ----------------------------------------------------------------------------- #
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def host_cores() -> int:
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return min(n, 64)   # OpenBLAS build limit (MAX_THREADS=64)
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "activation_sparse_ffn_predict_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel_key: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it matches the source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_sha") != source_sha():
+        return None
+    return rec.get("kernels", {}).get(kernel_key)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(pw) if pw else None}
+
+
+# ----------------------------------------------------------------------------- #
+# CPU oracle timing (reference arm and cpu_baseline)                            #
+# ----------------------------------------------------------------------------- #
+def oracle_items(cfg, B: int):
+    """Sampled (layer, token batch) items of the workload: first, middle and last layer."""
+    import synthetic as S
+    L = cfg.layers
+    layers = sorted({0, L // 2, L - 1})
+    prepared = []
+    for l in layers:
+        w = S.layer_weights(cfg, l, "cpu")
+        X = S.layer_tokens(cfg, l, 4 * B, "cpu").numpy()
+        prepared.append((l, w.numpy(), X))
+    return prepared, layers
+
+
+def oracle_layer_token_seconds(cfg, prepared, B: int, mode: str, budget_s: float, max_items=None):
+    """Time the oracle on the prepared items until the budget or item cap is reached."""
+    import oracle as O
+    items, t_total, k = 0, 0.0, 0
+    while True:
+        l, h, X = prepared[k % len(prepared)]
+        j = (k // len(prepared)) % 4
+        xb = X[j * B:(j + 1) * B]
+        t0 = time.perf_counter()
+        if mode == "dense":
+            O.dense_ffn(h["act"], h["Wg"], h["Wu"], h["WdT"], h["bias"], xb)
+        else:
+            idx, _ = O.predict(h["W1"], h["b1"], h["W2"], h["b2"], xb, cfg.tau)
+            O.sparse_ffn(h["act"], h["Wg"], h["Wu"], h["WdT"], h["bias"], xb, idx)
+        t_total += time.perf_counter() - t0
+        items += 1
+        k += 1
+        if t_total >= budget_s or (max_items is not None and items >= max_items):
+            break
+    return t_total / items, items
+
+
+def cpu_baseline(cfg, B, mode, seconds):
+    prepared, layers = oracle_items(cfg, B)
+    per_item, items = oracle_layer_token_seconds(cfg, prepared, B, mode, seconds)
+    value = B / (per_item * cfg.layers)
+    return {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+            "sample": (f"float64 NumPy oracle ({'dense FFN' if mode == 'dense' else 'predictor + sparse FFN'})"
+                       f" on {items} (layer, {B}-token batch) items drawn from layers {layers} of the "
+                       f"{cfg.layers}-layer stack, {per_item * 1e3:.1f} ms per item, scaled by "
+                       f"{cfg.layers} layers per step")}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    # each timed step is a bounded sample: one (layer, batch) item, scaled by L
+    prepared, layers = oracle_items(cfg, args.batch)
+    W = min(args.warmup, 2)
+    if W:
+        oracle_layer_token_seconds(cfg, prepared, args.batch, args.mode, 0.0, max_items=W)
+    per_item_est, _ = oracle_layer_token_seconds(cfg, prepared, args.batch, args.mode, 0.0, max_items=1)
+    k_fit = max(1, int(args.reference_budget / max(per_item_est, 1e-6)))
+    K = min(args.steps, k_fit)
+    per_item, items = oracle_layer_token_seconds(cfg, prepared, args.batch, args.mode, float("inf"),
+                                                 max_items=K)
+    step_s = per_item * cfg.layers
+    value = args.batch / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "steps_timed": items, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg, args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                         "sample": (f"{items} timed steps of the {args.steps} requested, each one "
+                                    f"(layer, {args.batch}-token batch) item from layers {layers}, "
+                                    f"scaled by {cfg.layers} layers")},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cfg, args):
+    hot = cfg.hot_perm and not args.no_hot_perm
+    return {"workload": (f"{cfg.name}: {cfg.layers} layers, d={cfg.d}, d_ffn={cfg.n}, predictor "
+                         f"{cfg.d}->{cfg.r}->{cfg.n}, {cfg.act}, {cfg.dtype} weights, batch {args.batch}, "
+                         f"Zipf({cfg.gamma}) with {cfg.frac:.0%} mean activity, tau={cfg.tau}, "
+                         f"hot rows {'first' if hot else 'in id order'}, mode {args.mode}"),
+            "layers": cfg.layers, "batch": args.batch,
+            "tokens_cycled": args.tokens if args.tokens > 0 else cfg.tokens,
+            "weights": cfg.dtype, "accumulate": "f32",
+            "l2": "inputs larger than L2: every step streams rows of all layers of a stack "
+                  "whose weights exceed the 126 MB L2 many times over",
+            "parallelism": f"replicas x{args.gpus}"}
+
+
+# ----------------------------------------------------------------------------- #
+# GPU arm                                                                       #
+# ----------------------------------------------------------------------------- #
+def hot_permute_layer(cfg, layer, w, device):
+    """Offline hot-neuron permutation through the library: counts, sort, gather."""
+    import torch
+    import synthetic as S
+    import activation_sparse_ffn_predict_b200 as A
+    ffn = A.FFN(w.act, w.Wg, w.Wu, w.WdT, w.bias)
+    ws = A.Workspace(None, ffn, 1, device=device)
+    Xc = S.layer_tokens(cfg, layer, cfg.calib_tokens, device, kind="x_calib")
+    counts = torch.zeros(cfg.n, dtype=torch.int64, device=device)
+    A.asf_activation_counts(ffn, Xc, counts, ws)
+    c = counts.cpu().numpy()
+    perm = A.asf_hot_permutation(c)
+    perm_d = torch.from_numpy(perm).to(device)
+
+    def prow(t):
+        if t is None:
+            return None
+        out = torch.empty_like(t)
+        A.asf_permute_rows(t, out, perm_d)
+        return out
+
+    new = type(w)(w.act, w.dtype, prow(w.Wg), prow(w.Wu), prow(w.WdT), prow(w.bias), w.W1, w.b1,
+                  prow(w.W2), prow(w.b2), w.p[perm])
+    torch.cuda.synchronize()
+    k_hot = int(cfg.n * cfg.hot_ratio)
+    share = float(c[perm[:k_hot]].sum()) / max(1, int(c.sum()))
+    return new, share
+
+
+def run_ours(args, cfg):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import synthetic as S
+    from activation_sparse_ffn_predict_b200 import build as _build
+    _build.build()
+    import activation_sparse_ffn_predict_b200 as A
+    from activation_sparse_ffn_predict_b200.stack import LayerStack, build_layers
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    B = args.batch
+    L = cfg.layers
+    T = args.tokens if args.tokens > 0 else cfg.tokens
+    hot = cfg.hot_perm and not args.no_hot_perm
+    weights, shares = [], []
+    for l in range(L):
+        w = S.layer_weights(cfg, l, device=device)
+        if hot:
+            w, share = hot_permute_layer(cfg, l, w, device)
+            shares.append(share)
+        weights.append(w)
+    preds, ffns = build_layers(weights, device)
+    st = LayerStack(preds, ffns, B, cfg.tau, mode=args.mode, device=device)
+    # token stream: each rank decodes its own tokens (replicas; no collectives)
+    X = torch.empty(T, L, B, cfg.d, dtype=st.dtype, device=device)
+    for l in range(L):
+        xl = S.layer_tokens(cfg, l, T * B * world, device)[rank * T * B:(rank + 1) * T * B]
+        X[:, l] = xl.reshape(T, B, cfg.d)
+
+    if args.mode == "sparse":
+        # sparse-only: the predictor's lists computed once, outside the timed region
+        idx_all = torch.empty(T, L, cfg.n, dtype=torch.int32, device=device)
+        cnt_all = torch.empty(T, L, dtype=torch.int32, device=device)
+        pst = LayerStack(preds, ffns, B, cfg.tau, mode="predict", device=device)
+        for t in range(T):
+            pst.x.copy_(X[t])
+            pst.step()
+            idx_all[t].copy_(pst.idx)
+            cnt_all[t].copy_(pst.count)
+        del pst
+
+    st.capture()
+
+    def step(i):
+        t = i % T
+        st.x.copy_(X[t], non_blocking=True)
+        if args.mode == "sparse":
+            st.idx.copy_(idx_all[t], non_blocking=True)
+            st.count.copy_(cnt_all[t], non_blocking=True)
+        st.step()
+
+    # active counts per (token, layer), for the touched-byte accounting
+    counts = np.zeros((T, L), dtype=np.int64)
+    if args.mode == "dense":
+        counts[:] = cfg.n
+    else:
+        for t in range(T):
+            step(t)
+            counts[t] = st.count.cpu().numpy()
+    torch.cuda.synchronize()
+
+    s = cfg.elem_bytes
+    m = cfg.mats
+    ffn_bytes_tl = counts * (m * cfg.d * s + 4)                         # per (token, layer)
+    pred_bytes_l = (cfg.r * cfg.d + cfg.n * cfg.r) * s + 4 * (cfg.r + cfg.n)
+    tok_seq = np.arange(args.steps) % T
+    ffn_bytes_step = float(ffn_bytes_tl[tok_seq].sum(axis=1).mean())
+    pred_bytes_step = float(pred_bytes_l * L) if args.mode == "predict" else 0.0
+
+    # ---------------------------------------------------------- timed region --
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier()
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.2)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(args.steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if rank == 0 else None
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    err = A.asf_read_error(st.ws)
+    if err != 0:
+        raise RuntimeError(f"device error during the timed region: {A.asf_status_string(err)}")
+    step_ms = ms / args.steps
+    value = args.steps * B * world / (ms / 1e3)
+
+    # ------------------------------------------------ per-call event timing --
+    # A second graph brackets each library call with timing events (the events
+    # cut the overlap between calls, so each call is timed on its own).
+    cap_stream = torch.cuda.Stream(device=device)
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(L)]
+    pst_mode = args.mode
+    g2 = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g2, stream=cap_stream):
+        for l in range(L):
+            x, y, cnt = st.x[l], st.y[l], st.count[l:l + 1]
+            ev[l][0].record()
+            if pst_mode == "predict":
+                A.asf_predict(st.preds[l], x, st.tau, st.idx[l], cnt, st.ws)
+            ev[l][1].record()
+            if pst_mode == "dense":
+                A.asf_dense_ffn(st.ffns[l], x, y, st.ws)
+            else:
+                A.asf_sparse_ffn(st.ffns[l], x, st.idx[l], cnt, y, st.ws)
+            ev[l][2].record()
+    torch.cuda.synchronize()
+    pred_ms, ffn_ms = [], []
+    nprof = min(args.profile_steps, T)
+    ffn_bytes_prof = 0.0
+    for i in range(nprof):
+        t = i % T
+        st.x.copy_(X[t])
+        if args.mode == "sparse":
+            st.idx.copy_(idx_all[t])
+            st.count.copy_(cnt_all[t])
+        g2.replay()
+        torch.cuda.synchronize()
+        for l in range(L):
+            pred_ms.append(ev[l][0].elapsed_time(ev[l][1]))
+            ffn_ms.append(ev[l][1].elapsed_time(ev[l][2]))
+        ffn_bytes_prof += float(ffn_bytes_tl[t].sum())
+    del g2
+    ffn_call_ms = max_over_ranks(float(np.mean(ffn_ms)))
+    ffn_gbs = (ffn_bytes_prof / (nprof * L)) / (ffn_call_ms * 1e-3) / 1e9
+    pred_call_ms = float(np.mean(pred_ms)) if args.mode == "predict" else 0.0
+    pred_gbs = pred_bytes_l / (pred_call_ms * 1e-3) / 1e9 if pred_call_ms > 0 else None
+
+    # -------------------------------------------------------------- e2e --------
+    Xh = X.cpu().pin_memory()
+    Yh = torch.empty(L, B, cfg.d, dtype=torch.float32).pin_memory()
+    ke = min(args.e2e_steps, args.steps)
+    for i in range(min(8, ke)):
+        st.x.copy_(Xh[i % T], non_blocking=True)
+        st.step()
+        Yh.copy_(st.y, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for i in range(ke):
+        t = i % T
+        st.x.copy_(Xh[t], non_blocking=True)
+        if args.mode == "sparse":
+            st.idx.copy_(idx_all[t], non_blocking=True)
+            st.count.copy_(cnt_all[t], non_blocking=True)
+        st.step()
+        Yh.copy_(st.y, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    f1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e_value = ke * B * world / (e2e_ms / 1e3)
+
+    st.release()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = measured_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    key = f"{cfg.name}:B{B}:{args.mode}"
+    tr = traffic_record(key)
+    roof = {"bound": "hbm", "kernel": ("sparse FFN call: k_ffn_gu + k_ffn_down"
+                                       if args.mode != "dense" else "dense FFN call: k_ffn_gu + k_ffn_down"),
+            "achieved": ffn_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": ffn_gbs / hbm_peak,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+            "frac_of_nominal_7700": ffn_gbs / NOMINAL_HBM_GBS,
+            "traffic": (tr["dram_bytes_per_launch"] if tr else None),
+            "algorithmic_bytes_per_launch": ffn_bytes_prof / (nprof * L),
+            "launch_ms": ffn_call_ms}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(cfg, args),
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(L * B * cfg.d * s),
+                "d2h_bytes_per_step": int(L * B * cfg.d * 4)},
+        "gpu_launches": int(args.steps * st.launches_per_step()),
+        "clocks": clocks,
+        "step_gbs": (ffn_bytes_step + pred_bytes_step) / (step_ms * 1e-3) / 1e9,
+        "touched_bytes_per_step": ffn_bytes_step + pred_bytes_step,
+        "active_per_layer_mean": float(counts[tok_seq].mean()),
+        "predictor_call": ({"ms": pred_call_ms, "gbs": pred_gbs, "frac": pred_gbs / hbm_peak,
+                            "bytes": pred_bytes_l} if pred_gbs else None),
+        "hot_share_top20": (float(np.mean(shares)) if shares else None),
+        "ideal_tokens_per_s_at_peak": hbm_peak * 1e9 / (ffn_bytes_step + pred_bytes_step) * B,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, B, args.mode, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    import synthetic as S
+    cfg = S.get(args.config)
+    if args.layers > 0:
+        cfg = cfg.with_(layers=args.layers)
+    if args.batch < 1 or args.batch > 32:
+        raise SystemExit("--batch must be in 1..32")
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

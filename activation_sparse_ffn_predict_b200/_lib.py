@@ -21,6 +21,7 @@ ASF_F16 = 1
 ASF_ACT_RELU = 0
 ASF_ACT_REGLU = 1
 ASF_MAX_BATCH = 32
+ASF_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class asf_predictor(ctypes.Structure):
@@ -47,6 +48,8 @@ PROTOTYPES = {
                                       c_size_t, c_void_p]),
     "asf_hot_permutation": (c_int, [POINTER(c_int64), c_int32, POINTER(c_int32)]),
     "asf_permute_rows": (c_int, [c_void_p, c_void_p, c_int32, c_int64, c_void_p, c_void_p]),
+    "asf_sparse_ffn_noalloc": (c_int, [POINTER(asf_ffn), c_void_p, c_int32, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p]),
     "asf_read_error": (c_int, [c_void_p, POINTER(c_int32), c_void_p]),
     "asf_status_string": (c_char_p, [c_int]),
     "asf_version": (c_int32, []),

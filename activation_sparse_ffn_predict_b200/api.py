@@ -136,6 +136,22 @@ def asf_sparse_ffn(ffn: FFN, x: torch.Tensor, idx: torch.Tensor, count: torch.Te
     check(st, "asf_sparse_ffn")
 
 
+def asf_sparse_ffn_noalloc(ffn: FFN, x: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
+                           y: torch.Tensor, fault: Optional[torch.Tensor] = None, stream=None) -> None:
+    """asf_sparse_ffn without a workspace: for callers that cannot allocate
+    device memory where they run the FFN (the library's own static device
+    scratch is used instead; calls that overlap on the GPU race)."""
+    if x.dtype != ffn.dtype or x.dim() != 2 or x.shape[1] != ffn.d:
+        raise ValueError("x must be [B, d] in the FFN's dtype")
+    if y.shape != (x.shape[0], ffn.d):
+        raise ValueError("y must be [B, d]")
+    fp = _dev(fault, "fault", torch.int32) if fault is not None else ctypes.c_void_p(0)
+    st = L.load().asf_sparse_ffn_noalloc(ctypes.byref(ffn.desc), _dev(x, "x"), int(x.shape[0]),
+                                         _dev(idx, "idx", torch.int32), _dev(count, "count", torch.int32),
+                                         _dev(y, "y", torch.float32), fp, _stream(stream))
+    check(st, "asf_sparse_ffn_noalloc")
+
+
 def asf_dense_ffn(ffn: FFN, x: torch.Tensor, y: torch.Tensor, ws: Workspace, stream=None) -> None:
     if x.dtype != ffn.dtype or x.dim() != 2 or x.shape[1] != ffn.d or y.shape != (x.shape[0], ffn.d):
         raise ValueError("x must be [B, d] in the FFN's dtype and y [B, d]")

@@ -1632,6 +1632,32 @@ asf_status counts_t(const asf_ffn *f, const void *x, int Ttok, int64_t *counts, 
 }  // namespace
 
 // ======================================================================== //
+// scratch for asf_sparse_ffn_noalloc                                       //
+// ======================================================================== //
+// File-scope device scratch used instead of a caller workspace.  In host code
+// the name is only a host-side stand-in; the device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ASF_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64] = {};
+
+asf_status noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ASF_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ASF_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ASF_OK;
+}
+}  // namespace
+
+// ======================================================================== //
 // C ABI                                                                    //
 // ======================================================================== //
 extern "C" {
@@ -1753,6 +1779,29 @@ asf_status asf_permute_rows(const void *src, void *dst, int32_t n_rows, int64_t 
   return cuda_status(launch(k_permute_rows, dim3(grid), dim3(kThreads), 0, (cudaStream_t)stream,
                             (const unsigned char *)src, (unsigned char *)dst, (int)n_rows, (long long)row_bytes,
                             perm, unit));
+}
+
+asf_status asf_sparse_ffn_noalloc(const asf_ffn *ffn, const void *x, int32_t B, const int32_t *idx,
+                                  const int32_t *count, float *y, int32_t *fault, asf_stream_t stream) {
+  asf_status s = check_ffn(ffn);
+  if (s != ASF_OK) return s;
+  if (!x || !idx || !count || !y) return ASF_ERR_INVALID_ARG;
+  if (B < 1 || B > ASF_MAX_BATCH) return ASF_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(y) || !al4(idx) || !al4(count) || (fault && !al4(fault))) return ASF_ERR_MISALIGNED;
+  const size_t need = kHeaderBytes + ffn_scratch(ffn, B);
+  if (need > (size_t)ASF_NOALLOC_SCRATCH_BYTES) return ASF_ERR_UNSUPPORTED;
+  void *ws = nullptr;
+  s = noalloc_scratch(&ws);
+  if (s != ASF_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  // counters and the fault word must start at zero; the rest is overwritten
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, st) != cudaSuccess) return ASF_ERR_CUDA;
+  s = ffn->wdtype == ASF_F16 ? ffn_t<__half>(ffn, x, B, idx, count, y, ws, st)
+                             : ffn_t<float>(ffn, x, B, idx, count, y, ws, st);
+  if (s != ASF_OK) return s;
+  if (fault && cudaMemcpyAsync(fault, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return ASF_ERR_CUDA;
+  return ASF_OK;
 }
 
 asf_status asf_read_error(void *ws, int32_t *host_out, asf_stream_t stream) {

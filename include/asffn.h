@@ -150,6 +150,33 @@ ASF_API asf_status asf_hot_permutation(const int64_t *counts, int32_t n, int32_t
 ASF_API asf_status asf_permute_rows(const void *src, void *dst, int32_t n_rows, int64_t row_bytes,
                             const int32_t *perm, asf_stream_t stream);
 
+/* Sparse FFN that allocates nothing and needs no workspace.
+ *
+ * No counterpart in the paper: this is a deployment convenience.  Some
+ * callers cannot allocate device memory where they run the FFN -- for example
+ * a plugin inside a host framework that owns every device allocation through
+ * its own pool, or a latency-critical path that cannot afford the implicit
+ * device synchronisation of cudaMalloc.  This call computes exactly what
+ * asf_sparse_ffn computes (same kernels), but takes its scratch from a
+ * file-scope device array of ASF_NOALLOC_SCRATCH_BYTES inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ *   ffn, x, B, idx, count, y   as for asf_sparse_ffn
+ *   fault   optional device int32: if not NULL, it receives the raw fault bits
+ *           of this call (0 = none; bit 0 = index out of range, bit 1 = timeout)
+ *
+ * The first call on each device looks up the array's device address for the
+ * current device (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  Each call clears the array's counters and fault word on `stream`
+ * before its kernels run.  All calls share the one array: calls that can
+ * overlap on the GPU (other streams, other threads) race and must be
+ * serialised by the caller.  Shapes whose scratch would exceed the array
+ * (larger d, n or B) return ASF_ERR_UNSUPPORTED without enqueuing anything.
+ * No device memory is allocated or freed, directly or by a library routine. */
+#define ASF_NOALLOC_SCRATCH_BYTES (8u << 20)
+ASF_API asf_status asf_sparse_ffn_noalloc(const asf_ffn *ffn, const void *x, int32_t B, const int32_t *idx,
+                                          const int32_t *count, float *y, int32_t *fault, asf_stream_t stream);
+
 /* Wait for the stream, then return (in *host_out) and clear the device error
  * word: 0, or the asf_status of the first device-side fault recorded. */
 ASF_API asf_status asf_read_error(void *ws, int32_t *host_out, asf_stream_t stream);

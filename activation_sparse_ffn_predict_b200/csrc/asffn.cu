@@ -22,7 +22,6 @@
 // Consecutive kernels overlap through programmatic dependent launch: each
 // kernel may prefetch its weights into L2 before waiting for its inputs.
 
-#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -30,9 +29,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
-#include <map>
 #include <mutex>
-#include <utility>
 #include <vector>
 
 #include "asffn.h"
@@ -48,9 +45,8 @@ constexpr int kMaxSplits = 64;        // max CTAs summing into one column tile
 constexpr int kTargetCtas = 296;      // 2 CTAs on each of the 148 SMs
 constexpr size_t kSmemBudget = 96 * 1024;
 constexpr int kFusedWarps = 8;        // consumer warps of the fused sparse FFN
-constexpr int kCluster = 8;           // CTAs per cluster (DSMEM reduction of y)
-constexpr int kMaxClusters = 32;      // partial-sum slots per column block
-constexpr size_t kFusedSmemDefault = 160 * 1024;
+constexpr int kMaxGrid = 256;         // upper bound of one-CTA-per-SM grids (partials, counts)
+constexpr size_t kFusedSmemDefault = 140 * 1024;
 constexpr uint64_t kWaitNs = 200ull * 1000 * 1000;  // bound on any mbarrier wait
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -471,12 +467,13 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
 }
 
 // Layer 2 + threshold + union + compaction, B <= NB tokens, with W2 rows fed
-// by the bulk-copy ring (first chunks issued before the wait).  Bits, ticket
-// and the last-CTA compaction are as in k_pred_l2.
+// by the bulk-copy ring (first chunks issued before the wait).  Each CTA keeps
+// the union bits of its rows in shared memory; after a grid barrier every CTA
+// writes its own part of the ascending list (one CTA per SM, all resident).
 template <typename T, int NB>
 __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
     k_pred2_ring(const T *__restrict__ W2, const float *__restrict__ b2, const float *__restrict__ h, int r, int n,
-                 int B, float thr, int rpc, int CR, int NSL, uint32_t *__restrict__ mask_words, int n_words,
+                 int B, float thr, int rpc, int CR, int NSL, int32_t *__restrict__ cta_counts,
                  int32_t *__restrict__ idx, int32_t *__restrict__ count, Header *__restrict__ hdr) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int V = Vec<T>::N;
@@ -488,7 +485,6 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
   float *hs = reinterpret_cast<float *>(smem + L.vec);
   uint32_t *smask = reinterpret_cast<uint32_t *>(smem + L.vec + (size_t)NB * r * 4);
   T *ring = reinterpret_cast<T *>(smem + L.ring);
-  __shared__ int s_last;
   __shared__ int s_wsum[NT / kWarp];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = blockIdx.x * rpc, row1 = min(n, row0 + rpc);
@@ -556,46 +552,42 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
       if (lane == 0) mbar_arrive(&empty[sl]);
     }
   }
+  // ---- distributed compaction: publish this CTA's count, meet the grid,
+  // then write this CTA's indices at its prefix offset (rows are contiguous
+  // per CTA and CTAs are in row order, so the result is ascending)
   __syncthreads();
-  for (int i = threadIdx.x; i < nwl; i += NT)
-    if (smask[i]) atomicOr(&mask_words[wfirst + i], smask[i]);
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = (ticket_acq_rel(&hdr->done) == gridDim.x - 1);
-  __syncthreads();
-  if (!s_last) return;
-  // ---- compaction by the last CTA: block-wide exclusive scan of popcounts ----
-  const int wpt = (n_words + NT - 1) / NT;
-  const int wbeg = min(n_words, (int)threadIdx.x * wpt);
-  const int wend = min(n_words, wbeg + wpt);
-  uint32_t wv[8];
   int local = 0;
-  for (int w = wbeg, q = 0; w < wend; ++w, ++q) {
-    const uint32_t m = ld_cg_u32(mask_words + w);
-    if (q < 8) wv[q] = m;
-    local += __popc(m);
-  }
-  int incl = local;
-#pragma unroll
-  for (int o = 1; o < kWarp; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == kWarp - 1) s_wsum[warp] = incl;
+  for (int i = 0; i < nwl; ++i) local += __popc(smask[i]);
+  if (threadIdx.x == 0) cta_counts[blockIdx.x] = local;
+  grid_barrier(hdr, gridDim.x, &hdr->err, kWaitNs);
+  int part_sum = 0;
+  for (int c = threadIdx.x; c < (int)blockIdx.x; c += NT) part_sum += ld_cg_i32(cta_counts + c);
+  part_sum = __reduce_add_sync(0xffffffffu, part_sum);
+  if (lane == 0) s_wsum[warp] = part_sum;
   __syncthreads();
-  int before = 0;
-  for (int w = 0; w < warp; ++w) before += s_wsum[w];
-  int off = before + incl - local;
-  for (int w = wbeg, q = 0; w < wend; ++w, ++q) {
-    uint32_t m = q < 8 ? wv[q] : ld_cg_u32(mask_words + w);
-    while (m) {
-      const int bit = __ffs(m) - 1;
-      idx[off++] = w * 32 + bit;
-      m &= m - 1u;
+  int offset = 0;
+  for (int w = 0; w < NT / kWarp; ++w) offset += s_wsum[w];
+  if (warp == 0) {
+    int base = offset;
+    for (int i0 = 0; i0 < nwl; i0 += kWarp) {
+      const int i = i0 + lane;
+      uint32_t m = i < nwl ? smask[i] : 0u;
+      const int pc = __popc(m);
+      int incl = pc;
+#pragma unroll
+      for (int o = 1; o < kWarp; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int off = base + incl - pc;
+      while (m) {
+        const int bit = __ffs(m) - 1;
+        idx[off++] = (wfirst + i) * 32 + bit;
+        m &= m - 1u;
+      }
+      base += __shfl_sync(0xffffffffu, incl, kWarp - 1);
     }
-  }
-  if (threadIdx.x == NT - 1) {
-    *count = off;
-    hdr->done = 0u;
+    if (lane == 0 && blockIdx.x == gridDim.x - 1) *count = offset + local;
   }
 }
 
@@ -779,7 +771,7 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ======================================================================== //
-// fused sparse FFN: bulk-copy ring + cluster reduction                     //
+// fused sparse FFN: bulk-copy ring + grid-barrier reduction                //
 // ======================================================================== //
 
 // Shared-memory layout of k_sparse_ffn for NS ring slots of M rows of d elements.
@@ -802,14 +794,7 @@ __host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int es
   L.x = o;     o += (size_t)NB * d * esz;
   o = align_up(o, 128);
   L.stage = o; o += (size_t)NS * M * d * esz;
-  const size_t red = (size_t)NB * d * 4;
-  if (red <= (size_t)NS * M * d * esz) {
-    L.red = L.stage;
-  } else {
-    o = align_up(o, 128);
-    L.red = o;
-    o += red;
-  }
+  L.red = 0;
   L.total = o;
   return L;
 }
@@ -826,21 +811,20 @@ __host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int es
 // shared memory, one named barrier, every warp sums the 8 partials in warp
 // order, applies ReLU(g + b) * u (or ReLU(u + b)), and accumulates
 // a * WdT[k] into its registers; then it releases the slot ("empty").
-// At the end the CTA's y partial is reduced across the cluster through DSMEM
-// (CTA rank q sums column block q in rank order) and across clusters by the
-// last cluster to finish each block (atomic ticket), in cluster order.
+// At the end every CTA stores its y partial, the grid meets at a bounded
+// barrier (all CTAs are resident: one per SM), and each CTA sums a slice of
+// columns over all partials in a fixed order -- deterministic, no float
+// atomics, and no single CTA finishing the work alone.
 template <typename T, int NB, int MAXQ, bool REGLU>
 __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     k_sparse_ffn(const T *__restrict__ Wg, const T *__restrict__ Wu, const T *__restrict__ WdT,
                  const float *__restrict__ bias, const T *__restrict__ x, int d, int n, int B,
                  const int32_t *__restrict__ idx, const int32_t *__restrict__ count, int NS,
                  float *__restrict__ part, float *__restrict__ y, Header *__restrict__ hdr) {
-  namespace cg = cooperative_groups;
   constexpr int V = Vec<T>::N;
   constexpr int M = REGLU ? 3 : 2;
   constexpr int NW = kFusedWarps;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_last;
   __shared__ int s_fail;
   const FusedLayout L = fused_layout(NS, d, M, (int)sizeof(T), NB);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
@@ -849,7 +833,6 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
   float *pd = reinterpret_cast<float *>(smem + L.pd);
   T *xs = reinterpret_cast<T *>(smem + L.x);
   T *stage = reinterpret_cast<T *>(smem + L.stage);
-  float *red = reinterpret_cast<float *>(smem + L.red);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nvec = d / V;
   const int grp = L.grp;
@@ -1024,65 +1007,59 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     }
     if (!ok) s_fail = 1;
   }
-  __syncthreads();
   // -------------------------------------------------------- reductions --
+  // this CTA's partial y, straight from registers (each lane owns its chunks)
   if (warp < NW) {
 #pragma unroll
     for (int qq = 0; qq < MAXQ; ++qq) {
       const int ch = (qq * NW + warp) * kWarp + lane;
       if (ch < nvec) {
 #pragma unroll
-        for (int b = 0; b < NB; ++b)
+        for (int b = 0; b < NB; ++b) {
+          if (b < B) {
+            float *dst = part + ((size_t)blockIdx.x * B + b) * d + (size_t)ch * V;
 #pragma unroll
-          for (int e = 0; e < V; ++e) red[(size_t)b * d + (size_t)ch * V + e] = acc[qq][e][b];
+            for (int e = 0; e < V; e += 4)
+              *reinterpret_cast<float4 *>(dst + e) =
+                  make_float4(acc[qq][e][b], acc[qq][e + 1][b], acc[qq][e + 2][b], acc[qq][e + 3][b]);
+          }
+        }
       }
     }
   }
-  cg::cluster_group cluster = cg::this_cluster();
-  cluster.sync();
-  const int crank = (int)cluster.block_rank();
-  const int ncl = G / kCluster;
-  const int cid = blockIdx.x / kCluster;
-  const int blk = ((nvec + kCluster - 1) / kCluster) * V;   // columns per block
-  const int c0 = min(d, crank * blk), c1 = min(d, c0 + blk);
+  grid_barrier(hdr, (unsigned)G, err, kWaitNs);
+  // CTA c sums columns [c0, c1) over the G partials: lanes split the partials,
+  // then a fixed xor-tree combines the lanes
+  const int cpb = (nvec + G - 1) / G;
+  const int c0 = min(d, blockIdx.x * cpb * V), c1 = min(d, c0 + cpb * V);
   const int w = c1 - c0;
-  const float *peer[kCluster];
+  // a warp takes up to 4 (token, column) items at once and issues all their
+  // loads before summing: one L2 round trip per 4 items
+  for (int it0 = warp * 4; it0 < B * w; it0 += (NW + 1) * 4) {
+    float v[4][8];
 #pragma unroll
-  for (int r = 0; r < kCluster; ++r) peer[r] = cluster.map_shared_rank(red, r);
-  for (int i = threadIdx.x; i < B * w; i += blockDim.x) {
-    const int b = i / w, col = c0 + (i - b * w);
-    float v[kCluster];
+    for (int k = 0; k < 4; ++k) {
+      const int it = it0 + k;
+      const int b = it < B * w ? it / w : 0, col = c0 + (it < B * w ? it - b * w : 0);
 #pragma unroll
-    for (int r = 0; r < kCluster; ++r) v[r] = peer[r][(size_t)b * d + col];
-    float sum = 0.f;
-#pragma unroll
-    for (int r = 0; r < kCluster; ++r) sum += v[r];
-    if (ncl == 1)
-      y[(size_t)b * d + col] = sum;
-    else
-      part[((size_t)cid * B + b) * d + col] = sum;
-  }
-  cluster.sync();
-  if (ncl == 1) return;
-  if (threadIdx.x == 0) s_last = (ticket_acq_rel(&hdr->tile_done[crank]) == (unsigned)ncl - 1u);
-  __syncthreads();
-  if (!s_last) return;
-  // all partials of an output are loaded before any is added (one L2 round
-  // trip, not one per cluster); the sum runs in cluster order
-  for (int i = threadIdx.x; i < B * w; i += blockDim.x) {
-    const int b = i / w, col = c0 + (i - b * w);
-    float sum = 0.f;
-    for (int q0 = 0; q0 < ncl; q0 += 4) {
-      float v[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) v[q] = q0 + q < ncl ? ld_cg_f32(part + ((size_t)(q0 + q) * B + b) * d + col) : 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (q0 + q < ncl) sum += v[q];
+      for (int u = 0; u < 8; ++u) {
+        const int q = lane + u * kWarp;
+        v[k][u] = (it < B * w && q < G) ? ld_cg_f32(part + ((size_t)q * B + b) * d + col) : 0.f;
+      }
     }
-    y[(size_t)b * d + col] = sum;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int it = it0 + k;
+      float sum = 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += v[k][u];
+      sum = warp_sum(sum);
+      if (lane == 0 && it < B * w) {
+        const int b = it / w, col = c0 + (it - b * w);
+        y[(size_t)b * d + col] = sum;
+      }
+    }
   }
-  if (threadIdx.x == 0) hdr->tile_done[crank] = 0u;
 }
 
 // ======================================================================== //
@@ -1219,70 +1196,6 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
-// Launch with a thread-block cluster of `cl` CTAs along x (plus PDL).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, int cl, cudaStream_t st,
-                           Args... args) {
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute((const void *)kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = cl;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
-
-// Clusters of `cl` CTAs that can be resident at once (cached per kernel/device).
-template <typename... KArgs>
-int max_clusters(void (*kern)(KArgs...), int threads, size_t smem, int cl) {
-  static std::mutex mu;
-  static std::map<std::pair<const void *, std::pair<int, size_t>>, int> cache;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  auto key = std::make_pair((const void *)kern, std::make_pair(dev, smem));
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
-  }
-  if (smem > 48 * 1024)
-    cudaFuncSetAttribute((const void *)kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(cl * 32);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cl;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, (const void *)kern, &cfg) != cudaSuccess || n <= 0) {
-    cudaGetLastError();
-    n = 0;
-  }
-  std::lock_guard<std::mutex> lk(mu);
-  cache[key] = n;
-  return n;
-}
-
 inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 inline size_t r256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -1298,12 +1211,13 @@ int down_splits(const asf_ffn *f) {
   return std::max(1, std::min(kMaxSplits, (kTargetCtas + ct - 1) / ct));
 }
 
-size_t pred_scratch(const asf_predictor *p, int B) {
-  return r256((size_t)n_words_of(p->n) * 4) + r256((size_t)B * p->r * 4);
+size_t mask_region(const asf_predictor *p) {
+  return r256((size_t)std::max(n_words_of(p->n), kMaxGrid) * 4);
 }
+size_t pred_scratch(const asf_predictor *p, int B) { return mask_region(p) + r256((size_t)B * p->r * 4); }
 size_t ffn_scratch(const asf_ffn *f, int B) {
   const size_t two_kernel = r256((size_t)f->n * B * 4) + r256((size_t)down_splits(f) * B * f->d * 4);
-  const size_t fused = r256((size_t)kMaxClusters * B * f->d * 4);
+  const size_t fused = r256((size_t)std::min(sm_count(), kMaxGrid) * B * f->d * 4);
   return std::max(two_kernel, fused);
 }
 
@@ -1409,8 +1323,9 @@ cudaError_t run_pred2_ring(const asf_predictor *p, int B, float thr, const float
   used = ring_shape((size_t)p->r * sizeof(T), vec, kRing2Smem, rpc, CR, NSL);
   if (!used) return cudaSuccess;
   const size_t smem = ring_layout(NSL, CR, p->r, (int)sizeof(T), vec).total;
+  int32_t *cta_counts = reinterpret_cast<int32_t *>(mask);   // counts live in the mask region
   return launch(k_pred2_ring<T, NB>, dim3(grid), dim3((kRingWarps + 1) * kWarp), smem, st, (const T *)p->W2,
-                p->b2, h, p->r, p->n, B, thr, rpc, CR, NSL, mask, n_words_of(p->n), idx, count, hdr);
+                p->b2, h, p->r, p->n, B, thr, rpc, CR, NSL, cta_counts, idx, count, hdr);
 }
 
 bool ring_enabled() {
@@ -1473,7 +1388,7 @@ asf_status predict_t(const asf_predictor *p, const void *x, int B, float thr, in
   unsigned char *base = static_cast<unsigned char *>(ws);
   Header *hdr = reinterpret_cast<Header *>(base);
   uint32_t *mask = reinterpret_cast<uint32_t *>(base + kHeaderBytes);
-  float *h = reinterpret_cast<float *>(base + kHeaderBytes + r256((size_t)n_words_of(p->n) * 4));
+  float *h = reinterpret_cast<float *>(base + kHeaderBytes + mask_region(p));
   const bool ring = B <= 8 && ring_enabled();
   bool used = false;
   cudaError_t e = cudaSuccess;
@@ -1518,6 +1433,10 @@ int fused_maxq(const asf_ffn *f) {
 }
 int fused_nb(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 0; }
 
+// One CTA per SM: every CTA is resident at once, which the grid barrier needs
+// (the ring's shared memory keeps a second CTA off each SM anyway).
+int fused_grid() { return std::min(sm_count(), kMaxGrid); }
+
 // Ring slots that fit the shared-memory budget (0 if fewer than two).
 int fused_slots(const asf_ffn *f, int NB) {
   const int M = f->act == ASF_ACT_REGLU ? 3 : 2;
@@ -1544,12 +1463,9 @@ cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *i
     const FusedLayout L = fused_layout(NS, f->d, M, (int)sizeof(T), NB);
     const int threads = (kFusedWarps + 1) * kWarp;
     auto kern = k_sparse_ffn<T, NB, MAXQ, REGLU>;
-    int ncl = max_clusters(kern, threads, L.total, kCluster);
-    ncl = std::min(ncl, std::min(kMaxClusters, (sm_count() + kCluster - 1) / kCluster));
-    if (ncl <= 0) return cudaErrorInvalidConfiguration;
-    return launch_cluster(kern, dim3(ncl * kCluster), dim3(threads), L.total, kCluster, st, (const T *)f->Wg,
-                          (const T *)f->Wu, (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count,
-                          NS, part, y, hdr);
+    const int G = fused_grid();
+    return launch(kern, dim3(G), dim3(threads), L.total, st, (const T *)f->Wg, (const T *)f->Wu,
+                  (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count, NS, part, y, hdr);
   }
 }
 

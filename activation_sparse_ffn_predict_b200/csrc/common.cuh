@@ -19,7 +19,10 @@ constexpr int kMaxTiles = 960;  // ticket slots for the down-projection reductio
 struct Header {
   int32_t err;
   uint32_t done;
-  uint32_t pad[14];
+  uint32_t bar_gen;        // grid barrier: number of barriers completed
+  uint32_t bar_top;        // grid barrier: groups arrived at the open barrier
+  uint32_t pad[12];
+  uint32_t bar_sub[32];    // grid barrier: CTAs arrived per group (0 between barriers)
   uint32_t tile_done[kMaxTiles];
 };
 static_assert(sizeof(Header) <= kHeaderBytes, "header too large");
@@ -72,18 +75,11 @@ __device__ __forceinline__ void fence_mbar_init() {
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t tx) {
-  uint64_t state;
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 %0, [%1], %2;"
-               : "=l"(state)
-               : "r"(smem_u32(bar)), "r"(tx)
-               : "memory");
-  (void)state;
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(tx) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  uint64_t state;
-  asm volatile("mbarrier.arrive.shared::cta.b64 %0, [%1];" : "=l"(state) : "r"(smem_u32(bar)) : "memory");
-  (void)state;
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
@@ -136,6 +132,56 @@ __device__ __forceinline__ uint32_t ticket_acq_rel(uint32_t *p) {
 
 __device__ __forceinline__ void flag_error(int32_t *err, int bit) {
   if (err) atomicOr(err, bit);
+}
+
+// Grid-wide barrier for a grid whose CTAs are all resident (one wave).
+// Arrival is two-level to keep atomic contention low: CTA c counts itself in
+// group c % G (G <= 16 groups); the last CTA of a group counts the group at
+// the top; the last group resets the counters and releases the next
+// generation.  Every other CTA polls the generation with acquire loads.  All
+// counters return to zero, so consecutive kernels may use different grid
+// sizes.  The wait is bounded: on timeout it records kErrTimeout and returns
+// false, and the kernel finishes without hanging (the workspace must then be
+// re-initialised).
+constexpr int kBarGroups = 16;
+__device__ __forceinline__ bool grid_barrier(Header *hdr, unsigned nctas, int32_t *err, uint64_t limit_ns) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned groups = nctas < (unsigned)kBarGroups ? nctas : (unsigned)kBarGroups;
+    const unsigned grp = blockIdx.x % groups;
+    const unsigned gsize = (nctas - grp + groups - 1) / groups;
+    uint32_t g0, old;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g0) : "l"(&hdr->bar_gen) : "memory");
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(&hdr->bar_sub[grp]) : "memory");
+    bool opened = false;
+    if (old == gsize - 1) {
+      asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(&hdr->bar_sub[grp]), "r"(0u) : "memory");
+      asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(&hdr->bar_top) : "memory");
+      if (old == groups - 1) {
+        asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(&hdr->bar_top), "r"(0u) : "memory");
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&hdr->bar_gen) : "memory");
+        opened = true;
+      }
+    }
+    int ok = 1;
+    if (!opened) {
+      const uint64_t t0 = global_ns();
+      for (;;) {
+        uint32_t g;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(&hdr->bar_gen) : "memory");
+        if (g != g0) break;
+        if (global_ns() - t0 > limit_ns) {
+          ok = 0;
+          flag_error(err, kErrTimeout);
+          break;
+        }
+      }
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -287,9 +287,9 @@ def run_ours(args, cfg):
     import activation_sparse_ffn_predict_b200 as A
     from activation_sparse_ffn_predict_b200.stack import LayerStack, build_layers
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from activation_sparse_ffn_predict_b200 import replicas as R
+    ri = R.RankInfo.from_env()
+    rank, world, local = ri.rank, ri.world, ri.local
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
@@ -299,16 +299,10 @@ def run_ours(args, cfg):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = R.barrier
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return R.max_over_ranks(v, device)
 
     B = args.batch
     L = cfg.layers
@@ -326,7 +320,7 @@ def run_ours(args, cfg):
     # token stream: each rank decodes its own tokens (replicas; no collectives)
     X = torch.empty(T, L, B, cfg.d, dtype=st.dtype, device=device)
     for l in range(L):
-        xl = S.layer_tokens(cfg, l, T * B * world, device)[rank * T * B:(rank + 1) * T * B]
+        xl = S.layer_tokens(cfg, l, T * B * world, device)[R.token_slice(rank, world, T * B)]
         X[:, l] = xl.reshape(T, B, cfg.d)
 
     if args.mode == "sparse":
@@ -394,7 +388,7 @@ def run_ours(args, cfg):
     if err != 0:
         raise RuntimeError(f"device error during the timed region: {A.asf_status_string(err)}")
     step_ms = ms / args.steps
-    value = args.steps * B * world / (ms / 1e3)
+    value = R.job_throughput(args.steps * B, world, ms)
 
     # ------------------------------------------------ per-call event timing --
     # A second graph brackets each library call with timing events (the events
@@ -464,7 +458,7 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1))
-    e2e_value = ke * B * world / (e2e_ms / 1e3)
+    e2e_value = R.job_throughput(ke * B, world, e2e_ms)
 
     st.release()
     if world > 1:

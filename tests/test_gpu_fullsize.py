@@ -1,0 +1,196 @@
+"""Parity at the workloads' full layer sizes, with the kernels and launch shapes
+the benchmark uses (the layer stack repeats these per-layer calls).
+
+For every configured model shape, sampled layers (first and last) are drawn on
+the device at full size.  The oracle then checks, one sampled output at a time:
+index lists for single tokens and for every configured batch union (bit-exact
+on conditioned predictor biases), the sparse FFN over the predicted lists, the
+dense FFN of one token through the true-active-set invariant, the offline
+activation counts of sampled rows, and the hot permutation.  The oracle reads
+only the rows it needs, gathered on the device and copied to the host.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synthetic as S
+from tests.gpu_util import ensure_built
+from tests.helpers import TOL, condition_b2, rel_err, relu_band_ambiguous
+
+import activation_sparse_ffn_predict_b200 as A
+
+pytestmark = pytest.mark.gpu
+
+FULL = ["llama2_7b_reglu", "falcon_40b_relu", "llama70b_reglu", "opt175b_relu"]
+N_TOK = 32
+
+
+class FullLayer:
+    def __init__(self, name, layer):
+        ensure_built()
+        cfg = S.get(name)
+        self.cfg = cfg
+        w = S.layer_weights(cfg, layer, device="cuda")
+        X = S.layer_tokens(cfg, layer, N_TOK, device="cuda")
+        self.Xh = X.cpu().numpy()
+        W1 = w.W1.cpu().numpy()
+        W2 = w.W2.cpu().numpy()
+        b1 = w.b1.cpu().numpy()
+        b2 = condition_b2(W1, b1, W2, w.b2.cpu().numpy(), self.Xh, cfg.tau)
+        w.b2 = torch.from_numpy(b2).cuda()
+        self.pred_host = (W1, b1, W2, b2)
+        self.w = w
+        self.X = X
+        self.pred = A.Predictor(w.W1, w.b1, w.W2, w.b2)
+        self.ffn = A.FFN(w.act, w.Wg, w.Wu, w.WdT, w.bias)
+        self.ws = A.Workspace(self.pred, self.ffn, 32)
+
+    def oracle_idx(self, rows):
+        W1, b1, W2, b2 = self.pred_host
+        return O.predict(W1, b1, W2, b2, self.Xh[rows], self.cfg.tau)[0]
+
+    def gathered(self, ids):
+        """Host copies of the rows the oracle needs, re-indexed 0..k-1."""
+        g = torch.from_numpy(np.asarray(ids, dtype=np.int64)).cuda()
+        take = lambda t: None if t is None else t.index_select(0, g).cpu().numpy()
+        return take(self.w.Wg), take(self.w.Wu), take(self.w.WdT), take(self.w.bias)
+
+    def oracle_y(self, rows, ids):
+        Wg, Wu, WdT, b = self.gathered(ids)
+        return O.sparse_ffn(self.cfg.act, Wg, Wu, WdT, b, self.Xh[rows], np.arange(len(ids)))
+
+
+_CACHE = {}
+
+
+@pytest.fixture(scope="module", params=[(n, l) for n in FULL for l in ("first", "last")],
+                ids=lambda p: f"{p[0]}-{p[1]}")
+def full_layer(request):
+    name, which = request.param
+    cfg = S.get(name)
+    layer = 0 if which == "first" else cfg.layers - 1
+    _CACHE.clear()
+    torch.cuda.empty_cache()
+    fl = FullLayer(name, layer)
+    yield fl
+    del fl
+    torch.cuda.empty_cache()
+
+
+def _batches(cfg):
+    return sorted(set(cfg.batches) | {1})
+
+
+def test_fullsize_predict_and_sparse_ffn(full_layer):
+    fl = full_layer
+    cfg = fl.cfg
+    for B in _batches(cfg):
+        starts = [0, 3] if B == 1 else [0]
+        for s0 in starts:
+            rows = slice(s0, s0 + B)
+            x = fl.X[rows].contiguous()
+            idx = torch.full((cfg.n,), -5, dtype=torch.int32, device="cuda")
+            cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+            y = torch.full((B, cfg.d), float("nan"), dtype=torch.float32, device="cuda")
+            A.asf_predict(fl.pred, x, cfg.tau, idx, cnt, fl.ws)
+            A.asf_sparse_ffn(fl.ffn, x, idx, cnt, y, fl.ws)
+            torch.cuda.synchronize()
+            c = int(cnt.item())
+            got = idx[:c].cpu().numpy()
+            ref = fl.oracle_idx(rows)
+            np.testing.assert_array_equal(got, ref)
+            yr = fl.oracle_y(rows, ref)
+            assert rel_err(y.cpu().numpy(), yr) <= TOL[cfg.dtype], (B, rel_err(y.cpu().numpy(), yr))
+    assert A.asf_read_error(fl.ws) == 0
+
+
+def test_fullsize_dense_equals_sparse_over_true_set(full_layer):
+    fl = full_layer
+    cfg = fl.cfg
+    if cfg.name not in ("opt175b_relu", "llama2_7b_reglu"):
+        pytest.skip("dense reference is part of the OPT-shaped workload (and the benchmark shape)")
+    rows = slice(5, 6)
+    x = fl.X[rows].contiguous()
+    y = torch.zeros(1, cfg.d, dtype=torch.float32, device="cuda")
+    A.asf_dense_ffn(fl.ffn, x, y, fl.ws)
+    torch.cuda.synchronize()
+    # true active set, computed by the oracle chunk by chunk over all rows
+    Wr = fl.w.Wg if cfg.act == "reglu" else fl.w.Wu
+    act = []
+    step = 4096
+    for s in range(0, cfg.n, step):
+        blk = Wr[s:s + step].cpu().numpy()
+        bb = fl.w.bias[s:s + step].cpu().numpy()
+        pre = O.relu_input("relu", None, blk, bb, fl.Xh[rows])[0]
+        act.append(np.flatnonzero(pre > 0) + s)
+    T = np.concatenate(act)
+    yr = fl.oracle_y(rows, T)
+    assert rel_err(y.cpu().numpy(), yr) <= TOL[cfg.dtype]
+
+
+def test_fullsize_activation_counts_and_permutation(full_layer):
+    fl = full_layer
+    cfg = fl.cfg
+    Xc = S.layer_tokens(cfg, 0, 256, device="cuda", kind="x_calib")
+    counts = torch.zeros(cfg.n, dtype=torch.int64, device="cuda")
+    A.asf_activation_counts(fl.ffn, Xc, counts, fl.ws)
+    torch.cuda.synchronize()
+    got = counts.cpu().numpy()
+    # sampled rows, each checked against the oracle within its rounding band
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(cfg.n, size=256, replace=False))
+    Wr = (fl.w.Wg if cfg.act == "reglu" else fl.w.Wu)
+    Wrows = Wr.index_select(0, torch.from_numpy(rows).cuda()).cpu().numpy()
+    brows = fl.w.bias.cpu().numpy()[rows]
+    Xn = Xc.cpu().numpy()
+    pre = O.relu_input("relu", None, Wrows, brows, Xn)
+    amb = relu_band_ambiguous("relu", None, Wrows, brows, Xn)
+    lo = ((pre > 0) & ~amb).sum(axis=0)
+    hi = ((pre > 0) | amb).sum(axis=0)
+    assert np.all(got[rows] >= lo) and np.all(got[rows] <= hi)
+    # the host permutation is the oracle's stable descending sort of these counts
+    perm = A.asf_hot_permutation(got)
+    np.testing.assert_array_equal(perm, O.hot_permutation(got))
+    # and the realised activity follows the configured profile (top 20% share)
+    _, _, share = O.partition(got, 0.2)
+    assert 0.6 < share < 0.85
+
+
+def test_fullsize_graph_stack_llama2_7b():
+    """Three full-size layers of the benchmark shape through the captured stack."""
+    ensure_built()
+    from activation_sparse_ffn_predict_b200.stack import LayerStack, build_layers
+    cfg = S.get("llama2_7b_reglu")
+    L = 3
+    ws, hosts, xs = [], [], []
+    for l in range(L):
+        w = S.layer_weights(cfg, l, device="cuda")
+        X = S.layer_tokens(cfg, l, 4, device="cuda")
+        W1, W2 = w.W1.cpu().numpy(), w.W2.cpu().numpy()
+        b2 = condition_b2(W1, w.b1.cpu().numpy(), W2, w.b2.cpu().numpy(), X.cpu().numpy(), cfg.tau)
+        w.b2 = torch.from_numpy(b2).cuda()
+        ws.append(w)
+        hosts.append((W1, w.b1.cpu().numpy(), W2, b2))
+        xs.append(X)
+    preds, ffns = build_layers(ws, "cuda")
+    st = LayerStack(preds, ffns, 1, cfg.tau, mode="predict")
+    st.capture()
+    for t in range(2):
+        for l in range(L):
+            st.x[l].copy_(xs[l][t:t + 1])
+        st.step()
+        torch.cuda.synchronize()
+        for l in range(L):
+            W1, b1, W2, b2 = hosts[l]
+            Xl = xs[l][t:t + 1].cpu().numpy()
+            ref = O.predict(W1, b1, W2, b2, Xl, cfg.tau)[0]
+            c = int(st.count[l].item())
+            np.testing.assert_array_equal(st.idx[l, :c].cpu().numpy(), ref)
+            g = torch.from_numpy(ref.astype(np.int64)).cuda()
+            take = lambda tt: tt.index_select(0, g).cpu().numpy()
+            yr = O.sparse_ffn("reglu", take(ws[l].Wg), take(ws[l].Wu), take(ws[l].WdT), take(ws[l].bias),
+                              Xl, np.arange(ref.size))
+            assert rel_err(st.y[l].cpu().numpy(), yr) <= TOL[cfg.dtype]
+    assert A.asf_read_error(st.ws) == 0
+    st.release()

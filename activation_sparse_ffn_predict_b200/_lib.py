@@ -31,7 +31,8 @@ class asf_predictor(ctypes.Structure):
 
 class asf_ffn(ctypes.Structure):
     _fields_ = [("d", c_int32), ("n", c_int32), ("wdtype", c_int), ("act", c_int),
-                ("Wg", c_void_p), ("Wu", c_void_p), ("WdT", c_void_p), ("bias", c_void_p)]
+                ("Wg", c_void_p), ("Wu", c_void_p), ("WdT", c_void_p), ("bias", c_void_p),
+                ("hot_rows", c_int32)]
 
 
 # name -> (restype, argtypes), exactly the declarations of include/asffn.h

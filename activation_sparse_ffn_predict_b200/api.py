@@ -59,7 +59,7 @@ class FFN:
     """Descriptor of one FFN layer in storage order: Wg/Wu/WdT [n,d], bias [n]."""
 
     def __init__(self, act: str, Wg: Optional[torch.Tensor], Wu: torch.Tensor, WdT: torch.Tensor,
-                 bias: torch.Tensor):
+                 bias: torch.Tensor, hot_rows: int = 0):
         if act not in _ACT:
             raise ValueError("act must be 'reglu' or 'relu'")
         if Wu.dtype not in _DT or WdT.dtype != Wu.dtype:
@@ -75,8 +75,9 @@ class FFN:
             gp = ctypes.c_void_p(0)
         self.tensors = (Wg, Wu, WdT, bias)
         self.act, self.d, self.n, self.dtype = act, d, n, Wu.dtype
+        self.hot_rows = int(hot_rows)
         self.desc = L.asf_ffn(d, n, _DT[Wu.dtype], _ACT[act], gp, _dev(Wu, "Wu"), _dev(WdT, "WdT"),
-                              _dev(bias, "bias", torch.float32))
+                              _dev(bias, "bias", torch.float32), self.hot_rows)
 
 
 def asf_version() -> int:

@@ -466,15 +466,14 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
   }
 }
 
-// Layer 2 + threshold + union + compaction, B <= NB tokens, with W2 rows fed
-// by the bulk-copy ring (first chunks issued before the wait).  Each CTA keeps
-// the union bits of its rows in shared memory; after a grid barrier every CTA
-// writes its own part of the ascending list (one CTA per SM, all resident).
+// Layer 2 + threshold + union over tokens, B <= NB tokens, with W2 rows fed by
+// the bulk-copy ring (first chunks issued before the wait).  Each CTA ORs the
+// bits of its rows into the union mask; the next kernel compacts it.
 template <typename T, int NB>
 __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
     k_pred2_ring(const T *__restrict__ W2, const float *__restrict__ b2, const float *__restrict__ h, int r, int n,
-                 int B, float thr, int rpc, int CR, int NSL, int32_t *__restrict__ cta_counts,
-                 int32_t *__restrict__ idx, int32_t *__restrict__ count, Header *__restrict__ hdr) {
+                 int B, float thr, int rpc, int CR, int NSL, uint32_t *__restrict__ mask_words,
+                 Header *__restrict__ hdr) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int V = Vec<T>::N;
   constexpr int NT = (kRingWarps + 1) * kWarp;
@@ -485,7 +484,6 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
   float *hs = reinterpret_cast<float *>(smem + L.vec);
   uint32_t *smask = reinterpret_cast<uint32_t *>(smem + L.vec + (size_t)NB * r * 4);
   T *ring = reinterpret_cast<T *>(smem + L.ring);
-  __shared__ int s_wsum[NT / kWarp];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = blockIdx.x * rpc, row1 = min(n, row0 + rpc);
   const int nch = row0 < row1 ? (row1 - row0 + CR - 1) / CR : 0;
@@ -521,6 +519,31 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
     }
     named_sync(1, kRingWarps * kWarp);
     const int nvec = r / V;
+    // A lane meets the same chunks of h in every row: keep them in registers
+    // when they fit (up to HQ chunks per lane, at most 2 tokens).
+    constexpr int HQ = 4;
+    constexpr bool kRegH = NB <= 2;
+    const bool reg_h = kRegH && nvec <= HQ * kWarp;
+    float hreg[kRegH ? NB : 1][HQ][V];
+    if (reg_h) {
+#pragma unroll
+      for (int b = 0; b < (kRegH ? NB : 1); ++b)
+#pragma unroll
+        for (int u = 0; u < HQ; ++u) {
+          const int c = lane + u * kWarp;
+#pragma unroll
+          for (int e = 0; e < V; ++e) {
+            float v = 0.f;
+            if (c < nvec) {
+              if constexpr (sizeof(T) == 2)
+                v = hs[(size_t)b * r + (e < 4 ? c * 4 + e : r / 2 + c * 4 + (e - 4))];
+              else
+                v = hs[(size_t)b * r + c * 4 + e];
+            }
+            hreg[b][u][e] = v;
+          }
+        }
+    }
     bool ok = true;
     for (int i = 0; i < nch; ++i) {
       const int sl = i % NSL;
@@ -534,10 +557,22 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
         float acc[NB];
 #pragma unroll
         for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-        for (int c = lane; c < nvec; c += kWarp) {
-          const uint4 wv = *reinterpret_cast<const uint4 *>(wr + (size_t)c * V);
+        if (reg_h) {
 #pragma unroll
-          for (int b = 0; b < NB; ++b) acc[b] += dot_hidden<T>(wv, hs + (size_t)b * r, r, c);
+          for (int u = 0; u < HQ; ++u) {
+            const int c = lane + u * kWarp;
+            if (c < nvec) {
+              const uint4 wv = *reinterpret_cast<const uint4 *>(wr + (size_t)c * V);
+#pragma unroll
+              for (int b = 0; b < (kRegH ? NB : 1); ++b) acc[b] = Vec<T>::dotr(wv, hreg[b][u], acc[b]);
+            }
+          }
+        } else {
+          for (int c = lane; c < nvec; c += kWarp) {
+            const uint4 wv = *reinterpret_cast<const uint4 *>(wr + (size_t)c * V);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) acc[b] += dot_hidden<T>(wv, hs + (size_t)b * r, r, c);
+          }
         }
         bool on = false;
         const float bias = __ldg(b2 + row);
@@ -552,43 +587,57 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
       if (lane == 0) mbar_arrive(&empty[sl]);
     }
   }
-  // ---- distributed compaction: publish this CTA's count, meet the grid,
-  // then write this CTA's indices at its prefix offset (rows are contiguous
-  // per CTA and CTAs are in row order, so the result is ascending)
+  // publish this CTA's union bits (words at the slice edges are shared with
+  // the neighbouring CTAs, hence the atomic OR); k_compact builds the list
   __syncthreads();
+  for (int i = threadIdx.x; i < nwl; i += NT)
+    if (smask[i]) atomicOr(&mask_words[wfirst + i], smask[i]);
+}
+
+// Ascending compaction of the union mask: one CTA reads every mask word,
+// scans the popcounts and writes the index list and its length.  A kernel
+// boundary is the cheapest grid-wide handoff on B200, so the scan runs as its
+// own small kernel right after the mask is complete.
+constexpr int kCompactThreads = 1024;
+constexpr int kCompactWords = 8;    // words per thread: n <= 1024 * 8 * 32
+__global__ void __launch_bounds__(kCompactThreads)
+    k_compact(const uint32_t *__restrict__ mask_words, int n_words, int32_t *__restrict__ idx,
+              int32_t *__restrict__ count) {
+  __shared__ int s_wsum[kCompactThreads / kWarp];
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wpt = (n_words + kCompactThreads - 1) / kCompactThreads;
+  const int wbeg = min(n_words, (int)threadIdx.x * wpt);
+  const int wend = min(n_words, wbeg + wpt);
+  uint32_t wv[kCompactWords];
   int local = 0;
-  for (int i = 0; i < nwl; ++i) local += __popc(smask[i]);
-  if (threadIdx.x == 0) cta_counts[blockIdx.x] = local;
-  grid_barrier(hdr, gridDim.x, &hdr->err, kWaitNs);
-  int part_sum = 0;
-  for (int c = threadIdx.x; c < (int)blockIdx.x; c += NT) part_sum += ld_cg_i32(cta_counts + c);
-  part_sum = __reduce_add_sync(0xffffffffu, part_sum);
-  if (lane == 0) s_wsum[warp] = part_sum;
-  __syncthreads();
-  int offset = 0;
-  for (int w = 0; w < NT / kWarp; ++w) offset += s_wsum[w];
-  if (warp == 0) {
-    int base = offset;
-    for (int i0 = 0; i0 < nwl; i0 += kWarp) {
-      const int i = i0 + lane;
-      uint32_t m = i < nwl ? smask[i] : 0u;
-      const int pc = __popc(m);
-      int incl = pc;
 #pragma unroll
-      for (int o = 1; o < kWarp; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      int off = base + incl - pc;
-      while (m) {
-        const int bit = __ffs(m) - 1;
-        idx[off++] = (wfirst + i) * 32 + bit;
-        m &= m - 1u;
-      }
-      base += __shfl_sync(0xffffffffu, incl, kWarp - 1);
-    }
-    if (lane == 0 && blockIdx.x == gridDim.x - 1) *count = offset + local;
+  for (int q = 0; q < kCompactWords; ++q) {
+    wv[q] = (wbeg + q < wend) ? ld_cg_u32(mask_words + wbeg + q) : 0u;
+    local += __popc(wv[q]);
   }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < kWarp; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == kWarp - 1) s_wsum[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += s_wsum[w];
+  int off = before + incl - local;
+#pragma unroll
+  for (int q = 0; q < kCompactWords; ++q) {
+    uint32_t m = wv[q];
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      idx[off++] = (wbeg + q) * 32 + bit;
+      m &= m - 1u;
+    }
+  }
+  if (threadIdx.x == kCompactThreads - 1) *count = off;
 }
 
 // ======================================================================== //
@@ -811,15 +860,13 @@ __host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int es
 // shared memory, one named barrier, every warp sums the 8 partials in warp
 // order, applies ReLU(g + b) * u (or ReLU(u + b)), and accumulates
 // a * WdT[k] into its registers; then it releases the slot ("empty").
-// At the end every CTA stores its y partial, the grid meets at a bounded
-// barrier (all CTAs are resident: one per SM), and each CTA sums a slice of
-// columns over all partials in a fixed order -- deterministic, no float
-// atomics, and no single CTA finishing the work alone.
+// At the end every CTA stores its y partial; k_reduce_partials, the next
+// kernel, sums them in a fixed order (deterministic, no float atomics).
 template <typename T, int NB, int MAXQ, bool REGLU>
 __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     k_sparse_ffn(const T *__restrict__ Wg, const T *__restrict__ Wu, const T *__restrict__ WdT,
                  const float *__restrict__ bias, const T *__restrict__ x, int d, int n, int B,
-                 const int32_t *__restrict__ idx, const int32_t *__restrict__ count, int NS,
+                 const int32_t *__restrict__ idx, const int32_t *__restrict__ count, int NS, int hot_rows,
                  float *__restrict__ part, float *__restrict__ y, Header *__restrict__ hdr) {
   constexpr int V = Vec<T>::N;
   constexpr int M = REGLU ? 3 : 2;
@@ -848,6 +895,21 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     s_fail = 0;
   }
   __syncthreads();
+  // Speculative warm-up: the leading hot_rows rows (hot neurons stored first)
+  // are active for most tokens, so their gate/up/down rows go to L2 while the
+  // predictor is still deciding; the bulk copies below then mostly hit L2.
+  if (hot_rows > 0 && warp == NW) {
+    const size_t bytes = (size_t)min(hot_rows, n) * d * sizeof(T);
+    const size_t per = (bytes / gridDim.x + 15) & ~(size_t)15;
+    const size_t o0 = min(bytes, per * blockIdx.x), o1 = min(bytes, o0 + per);
+    const T *mats[3] = {REGLU ? Wg : Wu, Wu, WdT};
+#pragma unroll
+    for (int m = REGLU ? 0 : 1; m < 3; ++m) {
+      const unsigned char *base = reinterpret_cast<const unsigned char *>(mats[m]);
+      for (size_t o = o0 + (size_t)lane * 16384; o < o1; o += 32 * 16384)
+        prefetch_l2(base + o, (uint32_t)min((size_t)16384, o1 - o));
+    }
+  }
   // The next kernel only prefetches weights before it waits on this one.
   pdl_trigger();
   pdl_wait();
@@ -921,6 +983,16 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
       *reinterpret_cast<uint4 *>(xs + (size_t)b * d + (size_t)c * V) = v;
     }
     named_sync(1, NW * kWarp);
+    // each lane meets the same chunks of x for every neuron: keep them in registers
+    uint4 xr[MAXQ][NB];
+#pragma unroll
+    for (int qq = 0; qq < MAXQ; ++qq) {
+      const int ch = (qq * NW + warp) * kWarp + lane;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        xr[qq][b] = ch < nvec ? *reinterpret_cast<const uint4 *>(xs + (size_t)b * d + (size_t)ch * V)
+                              : make_uint4(0u, 0u, 0u, 0u);
+    }
     bool ok = true;
     for (int g0 = 0; g0 < nl; g0 += grp) {
       const int gn = min(grp, nl - g0);
@@ -945,9 +1017,8 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
               if constexpr (REGLU) wg = *reinterpret_cast<const uint4 *>(rg + (size_t)ch * V);
 #pragma unroll
               for (int b = 0; b < NB; ++b) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)b * d + (size_t)ch * V);
-                pu[b] = Vec<T>::dot(wu, xv, pu[b]);
-                if constexpr (REGLU) pg[b] = Vec<T>::dot(wg, xv, pg[b]);
+                pu[b] = Vec<T>::dot(wu, xr[qq][b], pu[b]);
+                if constexpr (REGLU) pg[b] = Vec<T>::dot(wg, xr[qq][b], pg[b]);
               }
             }
           }
@@ -1027,38 +1098,40 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
       }
     }
   }
-  grid_barrier(hdr, (unsigned)G, err, kWaitNs);
-  // CTA c sums columns [c0, c1) over the G partials: lanes split the partials,
-  // then a fixed xor-tree combines the lanes
-  const int cpb = (nvec + G - 1) / G;
-  const int c0 = min(d, blockIdx.x * cpb * V), c1 = min(d, c0 + cpb * V);
-  const int w = c1 - c0;
-  // a warp takes up to 4 (token, column) items at once and issues all their
-  // loads before summing: one L2 round trip per 4 items
-  for (int it0 = warp * 4; it0 < B * w; it0 += (NW + 1) * 4) {
-    float v[4][8];
+}
+
+// y[b][col] = sum over the G per-CTA partials, in a fixed order: lanes own 32
+// consecutive columns (coalesced loads), the 8 warps split the partials and
+// all of a warp's loads are issued before any is added; warp sums are then
+// combined in warp order.
+constexpr int kReduceWarps = 8;
+constexpr int kReduceMaxPerWarp = 32;   // G <= 256
+__global__ void __launch_bounds__(kReduceWarps * kWarp)
+    k_reduce_partials(const float *__restrict__ part, int G, int B, int d, float *__restrict__ y) {
+  __shared__ float red[kReduceWarps][kWarp];
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int col = blockIdx.x * kWarp + lane;
+  const int b = blockIdx.y;
+  const int per = (G + kReduceWarps - 1) / kReduceWarps;
+  const int q0 = warp * per;
+  float v[kReduceMaxPerWarp];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int it = it0 + k;
-      const int b = it < B * w ? it / w : 0, col = c0 + (it < B * w ? it - b * w : 0);
+  for (int u = 0; u < kReduceMaxPerWarp; ++u) {
+    const int q = q0 + u;
+    v[u] = (u < per && q < G && col < d) ? ld_cg_f32(part + ((size_t)q * B + b) * d + col) : 0.f;
+  }
+  float s = 0.f;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int q = lane + u * kWarp;
-        v[k][u] = (it < B * w && q < G) ? ld_cg_f32(part + ((size_t)q * B + b) * d + col) : 0.f;
-      }
-    }
+  for (int u = 0; u < kReduceMaxPerWarp; ++u) s += v[u];
+  red[warp][lane] = s;
+  __syncthreads();
+  if (warp == 0 && col < d) {
+    float t = 0.f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int it = it0 + k;
-      float sum = 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) sum += v[k][u];
-      sum = warp_sum(sum);
-      if (lane == 0 && it < B * w) {
-        const int b = it / w, col = c0 + (it - b * w);
-        y[(size_t)b * d + col] = sum;
-      }
-    }
+    for (int w = 0; w < kReduceWarps; ++w) t += red[w][lane];
+    y[(size_t)b * d + col] = t;
   }
 }
 
@@ -1286,13 +1359,14 @@ cudaError_t run_pred_l2(const asf_predictor *p, int B, float thr, const float *h
 
 constexpr size_t kRingChunk = 32 * 1024;    // bytes per bulk copy of a ring slot
 constexpr size_t kRing1Smem = 80 * 1024;     // layer-1 ring + x: fits beside the fused FFN
-constexpr size_t kRing2Smem = 140 * 1024;
+constexpr size_t kRing2Smem = 168 * 1024;
 
 // rows per chunk and slots for a ring over rows of row_bytes within budget
 bool ring_shape(size_t row_bytes, size_t vec_bytes, size_t budget, int rpc, int &CR, int &NSL) {
   CR = (int)std::max<size_t>(1, kRingChunk / row_bytes);
   CR = std::min(CR, std::max(1, rpc));
-  for (NSL = 4; NSL >= 2; --NSL)
+  const int chunks = (rpc + CR - 1) / CR;        // slots that would hold the whole slice
+  for (NSL = std::min(8, std::max(chunks, 2)); NSL >= 2; --NSL)
     if (ring_layout(NSL, CR, 1, (int)row_bytes, vec_bytes).total <= budget) return true;
   return false;
 }
@@ -1323,9 +1397,10 @@ cudaError_t run_pred2_ring(const asf_predictor *p, int B, float thr, const float
   used = ring_shape((size_t)p->r * sizeof(T), vec, kRing2Smem, rpc, CR, NSL);
   if (!used) return cudaSuccess;
   const size_t smem = ring_layout(NSL, CR, p->r, (int)sizeof(T), vec).total;
-  int32_t *cta_counts = reinterpret_cast<int32_t *>(mask);   // counts live in the mask region
+  (void)idx;
+  (void)count;
   return launch(k_pred2_ring<T, NB>, dim3(grid), dim3((kRingWarps + 1) * kWarp), smem, st, (const T *)p->W2,
-                p->b2, h, p->r, p->n, B, thr, rpc, CR, NSL, cta_counts, idx, count, hdr);
+                p->b2, h, p->r, p->n, B, thr, rpc, CR, NSL, mask, hdr);
 }
 
 bool ring_enabled() {
@@ -1389,7 +1464,7 @@ asf_status predict_t(const asf_predictor *p, const void *x, int B, float thr, in
   Header *hdr = reinterpret_cast<Header *>(base);
   uint32_t *mask = reinterpret_cast<uint32_t *>(base + kHeaderBytes);
   float *h = reinterpret_cast<float *>(base + kHeaderBytes + mask_region(p));
-  const bool ring = B <= 8 && ring_enabled();
+  const bool ring = B <= 8 && ring_enabled() && n_words_of(p->n) <= kCompactThreads * kCompactWords;
   bool used = false;
   cudaError_t e = cudaSuccess;
   if (ring) e = pred1_ring_any<T>(p, x, B, h, mask, &hdr->err, st, used);
@@ -1397,8 +1472,11 @@ asf_status predict_t(const asf_predictor *p, const void *x, int B, float thr, in
   if (e != cudaSuccess) return ASF_ERR_CUDA;
   used = false;
   if (ring) e = pred2_ring_any<T>(p, B, thr, h, mask, idx, count, hdr, st, used);
-  if (e == cudaSuccess && !used) e = pred2_reg_any<T>(p, B, thr, h, mask, idx, count, hdr, st);
-  return cuda_status(e);
+  if (e != cudaSuccess) return ASF_ERR_CUDA;
+  if (used)   // the ring kernel leaves the union mask; compact it
+    return cuda_status(launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t *)mask,
+                              n_words_of(p->n), idx, count));
+  return cuda_status(pred2_reg_any<T>(p, B, thr, h, mask, idx, count, hdr, st));
 }
 
 // ------------------------------------------------------------------- ffn --
@@ -1433,8 +1511,7 @@ int fused_maxq(const asf_ffn *f) {
 }
 int fused_nb(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 0; }
 
-// One CTA per SM: every CTA is resident at once, which the grid barrier needs
-// (the ring's shared memory keeps a second CTA off each SM anyway).
+// One CTA per SM (the ring's shared memory keeps a second one off each SM).
 int fused_grid() { return std::min(sm_count(), kMaxGrid); }
 
 // Ring slots that fit the shared-memory budget (0 if fewer than two).
@@ -1464,8 +1541,12 @@ cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *i
     const int threads = (kFusedWarps + 1) * kWarp;
     auto kern = k_sparse_ffn<T, NB, MAXQ, REGLU>;
     const int G = fused_grid();
-    return launch(kern, dim3(G), dim3(threads), L.total, st, (const T *)f->Wg, (const T *)f->Wu,
-                  (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count, NS, part, y, hdr);
+    cudaError_t e = launch(kern, dim3(G), dim3(threads), L.total, st, (const T *)f->Wg, (const T *)f->Wu,
+                           (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count, NS,
+                           idx ? std::max(0, f->hot_rows) : 0, part, y, hdr);
+    if (e != cudaSuccess) return e;
+    return launch(k_reduce_partials, dim3((f->d + kWarp - 1) / kWarp, B), dim3(kReduceWarps * kWarp), 0, st,
+                  (const float *)part, G, B, f->d, y);
   }
 }
 
@@ -1578,7 +1659,7 @@ asf_status noalloc_scratch(void **out) {
 // ======================================================================== //
 extern "C" {
 
-int32_t asf_version(void) { return 100; }
+int32_t asf_version(void) { return 101; }
 
 const char *asf_status_string(asf_status s) {
   switch (s) {

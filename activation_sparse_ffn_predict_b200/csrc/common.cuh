@@ -19,10 +19,7 @@ constexpr int kMaxTiles = 960;  // ticket slots for the down-projection reductio
 struct Header {
   int32_t err;
   uint32_t done;
-  uint32_t bar_gen;        // grid barrier: number of barriers completed
-  uint32_t bar_top;        // grid barrier: groups arrived at the open barrier
-  uint32_t pad[12];
-  uint32_t bar_sub[32];    // grid barrier: CTAs arrived per group (0 between barriers)
+  uint32_t pad[14];
   uint32_t tile_done[kMaxTiles];
 };
 static_assert(sizeof(Header) <= kHeaderBytes, "header too large");
@@ -134,56 +131,6 @@ __device__ __forceinline__ void flag_error(int32_t *err, int bit) {
   if (err) atomicOr(err, bit);
 }
 
-// Grid-wide barrier for a grid whose CTAs are all resident (one wave).
-// Arrival is two-level to keep atomic contention low: CTA c counts itself in
-// group c % G (G <= 16 groups); the last CTA of a group counts the group at
-// the top; the last group resets the counters and releases the next
-// generation.  Every other CTA polls the generation with acquire loads.  All
-// counters return to zero, so consecutive kernels may use different grid
-// sizes.  The wait is bounded: on timeout it records kErrTimeout and returns
-// false, and the kernel finishes without hanging (the workspace must then be
-// re-initialised).
-constexpr int kBarGroups = 16;
-__device__ __forceinline__ bool grid_barrier(Header *hdr, unsigned nctas, int32_t *err, uint64_t limit_ns) {
-  __shared__ int s_ok;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned groups = nctas < (unsigned)kBarGroups ? nctas : (unsigned)kBarGroups;
-    const unsigned grp = blockIdx.x % groups;
-    const unsigned gsize = (nctas - grp + groups - 1) / groups;
-    uint32_t g0, old;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g0) : "l"(&hdr->bar_gen) : "memory");
-    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(&hdr->bar_sub[grp]) : "memory");
-    bool opened = false;
-    if (old == gsize - 1) {
-      asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(&hdr->bar_sub[grp]), "r"(0u) : "memory");
-      asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(&hdr->bar_top) : "memory");
-      if (old == groups - 1) {
-        asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(&hdr->bar_top), "r"(0u) : "memory");
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&hdr->bar_gen) : "memory");
-        opened = true;
-      }
-    }
-    int ok = 1;
-    if (!opened) {
-      const uint64_t t0 = global_ns();
-      for (;;) {
-        uint32_t g;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(&hdr->bar_gen) : "memory");
-        if (g != g0) break;
-        if (global_ns() - t0 > limit_ns) {
-          ok = 0;
-          flag_error(err, kErrTimeout);
-          break;
-        }
-      }
-    }
-    s_ok = ok;
-  }
-  __syncthreads();
-  return s_ok != 0;
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -211,6 +158,13 @@ template <> struct Vec<float> {
     acc = fmaf(__uint_as_float(w.y), a.y, acc);
     acc = fmaf(__uint_as_float(w.z), a.z, acc);
     acc = fmaf(__uint_as_float(w.w), a.w, acc);
+    return acc;
+  }
+  __device__ __forceinline__ static float dotr(uint4 w, const float (&x)[4], float acc) {
+    acc = fmaf(__uint_as_float(w.x), x[0], acc);
+    acc = fmaf(__uint_as_float(w.y), x[1], acc);
+    acc = fmaf(__uint_as_float(w.z), x[2], acc);
+    acc = fmaf(__uint_as_float(w.w), x[3], acc);
     return acc;
   }
   __device__ __forceinline__ static void to_float(uint4 w, float (&f)[4]) {
@@ -249,6 +203,15 @@ template <> struct Vec<__half> {
     p = h2f(w.y); acc = fmaf(p.x, a.z, acc); acc = fmaf(p.y, a.w, acc);
     p = h2f(w.z); acc = fmaf(p.x, b.x, acc); acc = fmaf(p.y, b.y, acc);
     p = h2f(w.w); acc = fmaf(p.x, b.z, acc); acc = fmaf(p.y, b.w, acc);
+    return acc;
+  }
+  // acc + sum_i w_i * x_i with x as 8 floats held in registers
+  __device__ __forceinline__ static float dotr(uint4 w, const float (&x)[8], float acc) {
+    float2 p;
+    p = h2f(w.x); acc = fmaf(p.x, x[0], acc); acc = fmaf(p.y, x[1], acc);
+    p = h2f(w.y); acc = fmaf(p.x, x[2], acc); acc = fmaf(p.y, x[3], acc);
+    p = h2f(w.z); acc = fmaf(p.x, x[4], acc); acc = fmaf(p.y, x[5], acc);
+    p = h2f(w.w); acc = fmaf(p.x, x[6], acc); acc = fmaf(p.y, x[7], acc);
     return acc;
   }
   __device__ __forceinline__ static void to_float(uint4 w, float (&f)[8]) {

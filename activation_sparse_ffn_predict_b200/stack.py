@@ -78,10 +78,13 @@ class LayerStack:
         self.graph = None
 
 
-def build_layers(weights: List, device) -> tuple:
-    """Predictor and FFN descriptors for a list of ``synthetic.LayerWeights`` on ``device``."""
+def build_layers(weights: List, device, hot_rows: Optional[Sequence[int]] = None) -> tuple:
+    """Predictor and FFN descriptors for a list of ``synthetic.LayerWeights`` on ``device``.
+
+    hot_rows[l] (optional) is the number of leading rows of layer l that the
+    offline profile found active for most tokens (the prefetch hint)."""
     preds, ffns = [], []
-    for w in weights:
+    for l, w in enumerate(weights):
         preds.append(Predictor(w.W1, w.b1, w.W2, w.b2))
-        ffns.append(FFN(w.act, w.Wg, w.Wu, w.WdT, w.bias))
+        ffns.append(FFN(w.act, w.Wg, w.Wu, w.WdT, w.bias, hot_rows=(hot_rows[l] if hot_rows else 0)))
     return preds, ffns

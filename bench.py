@@ -43,6 +43,8 @@ def parse_args(argv=None):
     p.add_argument("--batch", type=int, default=1)
     p.add_argument("--mode", choices=["predict", "sparse", "dense"], default="predict")
     p.add_argument("--no-hot-perm", action="store_true", help="keep neuron id order")
+    p.add_argument("--no-hot-prefetch", action="store_true",
+                   help="do not pass the hot-row prefetch hint to the sparse FFN")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=1024)
@@ -273,7 +275,10 @@ def hot_permute_layer(cfg, layer, w, device):
     torch.cuda.synchronize()
     k_hot = int(cfg.n * cfg.hot_ratio)
     share = float(c[perm[:k_hot]].sum()) / max(1, int(c.sum()))
-    return new, share
+    # leading rows active for at least half of the calibration tokens: the
+    # prefetch hint the sparse FFN uses while the predictor runs
+    hot_rows = int((c[perm] * 2 >= cfg.calib_tokens).sum())
+    return new, share, hot_rows
 
 
 def run_ours(args, cfg):
@@ -308,14 +313,15 @@ def run_ours(args, cfg):
     L = cfg.layers
     T = args.tokens if args.tokens > 0 else cfg.tokens
     hot = cfg.hot_perm and not args.no_hot_perm
-    weights, shares = [], []
+    weights, shares, hot_rows = [], [], []
     for l in range(L):
         w = S.layer_weights(cfg, l, device=device)
         if hot:
-            w, share = hot_permute_layer(cfg, l, w, device)
+            w, share, hr = hot_permute_layer(cfg, l, w, device)
             shares.append(share)
+            hot_rows.append(0 if args.no_hot_prefetch else hr)
         weights.append(w)
-    preds, ffns = build_layers(weights, device)
+    preds, ffns = build_layers(weights, device, hot_rows if hot else None)
     st = LayerStack(preds, ffns, B, cfg.tau, mode=args.mode, device=device)
     # token stream: each rank decodes its own tokens (replicas; no collectives)
     X = torch.empty(T, L, B, cfg.d, dtype=st.dtype, device=device)
@@ -495,6 +501,7 @@ def run_ours(args, cfg):
         "predictor_call": ({"ms": pred_call_ms, "gbs": pred_gbs, "frac": pred_gbs / hbm_peak,
                             "bytes": pred_bytes_l} if pred_gbs else None),
         "hot_share_top20": (float(np.mean(shares)) if shares else None),
+        "hot_rows_mean": (float(np.mean(hot_rows)) if hot_rows else 0.0),
         "ideal_tokens_per_s_at_peak": hbm_peak * 1e9 / (ffn_bytes_step + pred_bytes_step) * B,
     }
     if not args.no_cpu_baseline:

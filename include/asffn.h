@@ -93,6 +93,10 @@ typedef struct {
   const void *Wu;     /* [n][d] up rows */
   const void *WdT;    /* [n][d] W_down transposed: row k = column k of W_down */
   const float *bias;  /* [n] bias of the ReLU input: gate (REGLU) or up (RELU) */
+  int32_t hot_rows;   /* rows 0..hot_rows-1 are active for most tokens (hot neurons stored
+                         first by the offline permutation); asf_sparse_ffn prefetches them
+                         into L2 while the list is still being predicted.  0 = no hint.
+                         Affects speed only, never results. */
 } asf_ffn;
 
 /* Bytes of device workspace needed by asf_predict / asf_sparse_ffn /
@@ -184,7 +188,7 @@ ASF_API asf_status asf_read_error(void *ws, int32_t *host_out, asf_stream_t stre
 /* Static description of a status code. */
 ASF_API const char *asf_status_string(asf_status s);
 
-/* ABI version: major * 100 + minor. */
+/* ABI version: major * 100 + minor (1.01 added asf_ffn.hot_rows). */
 ASF_API int32_t asf_version(void);
 
 #ifdef __cplusplus

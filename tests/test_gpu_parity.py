@@ -232,3 +232,24 @@ def test_permute_rows_unaligned_units():
     A.asf_permute_rows(src, dst, perm)
     torch.cuda.synchronize()
     assert torch.equal(dst.cpu(), src.cpu()[perm.cpu().long()])
+
+
+def test_hot_row_hint_changes_nothing_but_speed(layer):
+    cfg = layer.cfg
+    w = layer.w
+    hinted = A.FFN(w.act, w.Wg, w.Wu, w.WdT, w.bias, hot_rows=cfg.n // 2)
+    for B in (1, 3):
+        rows = slice(0, B)
+        idx = layer.oracle_idx(rows)
+        x = layer.Xd[rows].contiguous()
+        idt = torch.zeros(cfg.n, dtype=torch.int32, device="cuda")
+        if idx.size:
+            idt[:idx.size] = torch.from_numpy(idx).cuda()
+        cnt = torch.tensor([idx.size], dtype=torch.int32, device="cuda")
+        y0 = torch.zeros(B, cfg.d, dtype=torch.float32, device="cuda")
+        y1 = torch.zeros(B, cfg.d, dtype=torch.float32, device="cuda")
+        A.asf_sparse_ffn(layer.ffn, x, idt, cnt, y0, layer.ws)
+        A.asf_sparse_ffn(hinted, x, idt, cnt, y1, layer.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y0, y1)
+    assert layer.error() == 0

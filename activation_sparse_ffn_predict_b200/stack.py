@@ -40,8 +40,11 @@ class LayerStack:
         self.graph: Optional[torch.cuda.CUDAGraph] = None
 
     def launches_per_step(self) -> int:
-        """Kernels this library launches per step."""
-        return self.L * (4 if self.mode == "predict" else 2)
+        """Kernels this library launches per step: the predictor is two GEMV
+        kernels plus the compaction kernel for batches of up to 8 tokens (two
+        kernels otherwise); the sparse or dense FFN is two kernels."""
+        pred = (3 if self.B <= 8 else 2) if self.mode == "predict" else 0
+        return self.L * (pred + 2)
 
     def enqueue(self, stream=None) -> None:
         for l in range(self.L):

@@ -476,8 +476,9 @@ def run_ours(args, cfg):
     hbm_peak = float(peaks["hbm_gbs"])
     key = f"{cfg.name}:B{B}:{args.mode}"
     tr = traffic_record(key)
-    roof = {"bound": "hbm", "kernel": ("sparse FFN call: k_ffn_gu + k_ffn_down"
-                                       if args.mode != "dense" else "dense FFN call: k_ffn_gu + k_ffn_down"),
+    two = "k_sparse_ffn + k_reduce_partials" if B <= 4 else "k_ffn_gu + k_ffn_down"
+    roof = {"bound": "hbm", "kernel": f"{'dense' if args.mode == 'dense' else 'sparse'} FFN call ({two}), "
+                                      f"timed alone with CUDA events around each call in a captured graph",
             "achieved": ffn_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": ffn_gbs / hbm_peak,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
             "frac_of_nominal_7700": ffn_gbs / NOMINAL_HBM_GBS,

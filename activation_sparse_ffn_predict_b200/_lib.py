@@ -32,7 +32,7 @@ class asf_predictor(ctypes.Structure):
 class asf_ffn(ctypes.Structure):
     _fields_ = [("d", c_int32), ("n", c_int32), ("wdtype", c_int), ("act", c_int),
                 ("Wg", c_void_p), ("Wu", c_void_p), ("WdT", c_void_p), ("bias", c_void_p),
-                ("hot_rows", c_int32)]
+                ("hot_rows", c_int32), ("row_stride", c_int32)]
 
 
 # name -> (restype, argtypes), exactly the declarations of include/asffn.h
@@ -49,6 +49,8 @@ PROTOTYPES = {
                                       c_size_t, c_void_p]),
     "asf_hot_permutation": (c_int, [POINTER(c_int64), c_int32, POINTER(c_int32)]),
     "asf_permute_rows": (c_int, [c_void_p, c_void_p, c_int32, c_int64, c_void_p, c_void_p]),
+    "asf_gather_rows": (c_int, [c_void_p, c_int64, c_int32, c_void_p, c_int64, c_int32, c_int64, c_void_p,
+                                c_void_p]),
     "asf_sparse_ffn_noalloc": (c_int, [POINTER(asf_ffn), c_void_p, c_int32, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_void_p]),
     "asf_read_error": (c_int, [c_void_p, POINTER(c_int32), c_void_p]),

@@ -58,6 +58,28 @@ class Predictor:
 class FFN:
     """Descriptor of one FFN layer in storage order: Wg/Wu/WdT [n,d], bias [n]."""
 
+    @classmethod
+    def packed(cls, act: str, packed: torch.Tensor, bias: torch.Tensor, hot_rows: int = 0) -> "FFN":
+        """Layer in the neuron-major packed layout: packed[k] = [gate_k | up_k | down_k]
+        (ReGLU, shape [n, 3, d]) or [up_k | down_k] (ReLU, shape [n, 2, d])."""
+        if act not in _ACT or packed.dim() != 3 or packed.dtype not in _DT:
+            raise ValueError("packed must be [n, m, d] float16/float32")
+        n, m, d = packed.shape
+        if m != (3 if act == "reglu" else 2) or bias.shape != (n,):
+            raise ValueError("packed layer shape does not match the activation")
+        base = _dev(packed, "packed").value
+        rb = d * packed.element_size()
+        self = cls.__new__(cls)
+        self.tensors = (packed, bias)
+        self.act, self.d, self.n, self.dtype = act, d, n, packed.dtype
+        self.hot_rows = int(hot_rows)
+        gp = ctypes.c_void_p(base) if act == "reglu" else ctypes.c_void_p(0)
+        up = ctypes.c_void_p(base + (rb if act == "reglu" else 0))
+        dn = ctypes.c_void_p(base + (m - 1) * rb)
+        self.desc = L.asf_ffn(d, n, _DT[packed.dtype], _ACT[act], gp, up, dn,
+                              _dev(bias, "bias", torch.float32), self.hot_rows, m * d)
+        return self
+
     def __init__(self, act: str, Wg: Optional[torch.Tensor], Wu: torch.Tensor, WdT: torch.Tensor,
                  bias: torch.Tensor, hot_rows: int = 0):
         if act not in _ACT:
@@ -77,7 +99,7 @@ class FFN:
         self.act, self.d, self.n, self.dtype = act, d, n, Wu.dtype
         self.hot_rows = int(hot_rows)
         self.desc = L.asf_ffn(d, n, _DT[Wu.dtype], _ACT[act], gp, _dev(Wu, "Wu"), _dev(WdT, "WdT"),
-                              _dev(bias, "bias", torch.float32), self.hot_rows)
+                              _dev(bias, "bias", torch.float32), self.hot_rows, 0)
 
 
 def asf_version() -> int:
@@ -191,6 +213,38 @@ def asf_permute_rows(src: torch.Tensor, dst: torch.Tensor, perm: torch.Tensor, s
     st = L.load().asf_permute_rows(_dev(src, "src"), _dev(dst, "dst"), n_rows, row_bytes,
                                    _dev(perm, "perm", torch.int32), _stream(stream))
     check(st, "asf_permute_rows")
+
+
+def asf_gather_rows(src: torch.Tensor, dst: torch.Tensor, perm: Optional[torch.Tensor] = None, *,
+                    dst_offset: int = 0, dst_stride: Optional[int] = None, stream=None) -> None:
+    """Row gather on the device: row i of dst (dst_stride bytes apart, starting
+    dst_offset bytes into dst) = row perm[i] of src (identity without perm)."""
+    if src.dim() < 1 or src.shape[0] == 0:
+        raise ValueError("src needs at least one row")
+    src_rows = int(src.shape[0])
+    row_bytes = src.numel() * src.element_size() // src_rows
+    n_rows = int(perm.shape[0]) if perm is not None else src_rows
+    stride = int(dst_stride) if dst_stride is not None else row_bytes
+    need = dst_offset + (n_rows - 1) * stride + row_bytes if n_rows else 0
+    if dst_offset < 0 or stride < row_bytes or need > dst.numel() * dst.element_size():
+        raise ValueError("destination rows do not fit in dst")
+    pp = _dev(perm, "perm", torch.int32) if perm is not None else ctypes.c_void_p(0)
+    st = L.load().asf_gather_rows(_dev(src, "src"), row_bytes, src_rows,
+                                  ctypes.c_void_p(_dev(dst, "dst").value + dst_offset), stride, n_rows,
+                                  row_bytes, pp, _stream(stream))
+    check(st, "asf_gather_rows")
+
+
+def pack_layer(act: str, Wg: Optional[torch.Tensor], Wu: torch.Tensor, WdT: torch.Tensor,
+               perm: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Neuron-major packed copy [n, m, d] of a layer's rows (optionally permuted)."""
+    n, d = Wu.shape
+    mats = [Wg, Wu, WdT] if act == "reglu" else [Wu, WdT]
+    out = torch.empty(n, len(mats), d, dtype=Wu.dtype, device=Wu.device)
+    rb = d * Wu.element_size()
+    for m, W in enumerate(mats):
+        asf_gather_rows(W, out, perm, dst_offset=m * rb, dst_stride=len(mats) * rb, stream=stream)
+    return out
 
 
 def asf_read_error(ws: Workspace, stream=None) -> int:

@@ -121,12 +121,22 @@ template <typename T, int NB>
 __device__ __forceinline__ void stage_tokens(T *xs, const T *__restrict__ x, int d, int g0, int nb) {
   constexpr int V = Vec<T>::N;
   const int nvec = d / V;
-  for (int i = threadIdx.x; i < NB * nvec; i += blockDim.x) {
-    const int b = i / nvec;
-    const int c = i - b * nvec;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (b < nb) v = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)(g0 + b) * d + (size_t)c * V));
-    *reinterpret_cast<uint4 *>(xs + (size_t)b * d + (size_t)c * V) = v;
+  constexpr int MAXU = 4;    // loads issued before the first store
+  for (int i0 = threadIdx.x; i0 < NB * nvec; i0 += MAXU * blockDim.x) {
+    uint4 v[MAXU];
+#pragma unroll
+    for (int u = 0; u < MAXU; ++u) {
+      const int i = i0 + u * blockDim.x;
+      const int b = i / nvec;
+      v[u] = (i < NB * nvec && b < nb)
+                 ? __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)(g0 + b) * d) + (i - b * nvec))
+                 : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < MAXU; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < NB * nvec) reinterpret_cast<uint4 *>(xs)[i] = v[u];
+    }
   }
 }
 
@@ -137,6 +147,27 @@ __device__ __forceinline__ void prefetch_range(const void *p, size_t bytes) {
   const unsigned char *c = static_cast<const unsigned char *>(p);
   for (size_t o = (size_t)threadIdx.x * kPiece; o < bytes; o += (size_t)blockDim.x * kPiece)
     prefetch_l2(c + o, (uint32_t)min(kPiece, bytes - o));
+}
+
+// Copy n16 16-byte units from global (data written by the previous kernel,
+// read through L2) into shared memory using the first `nthreads` threads.  All
+// of a thread's loads are issued before its first store, so the copy costs one
+// memory round trip instead of one per unit.
+template <int MAXU>
+__device__ __forceinline__ void stage16(uint4 *dst, const uint4 *__restrict__ src, int n16, int nthreads) {
+  if ((int)threadIdx.x >= nthreads) return;
+  uint4 v[MAXU];
+#pragma unroll
+  for (int u = 0; u < MAXU; ++u) {
+    const int i = threadIdx.x + u * nthreads;
+    v[u] = i < n16 ? __ldcg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int u = 0; u < MAXU; ++u) {
+    const int i = threadIdx.x + u * nthreads;
+    if (i < n16) dst[i] = v[u];
+  }
+  for (int i = threadIdx.x + MAXU * nthreads; i < n16; i += nthreads) dst[i] = __ldcg(src + i);
 }
 
 // ======================================================================== //
@@ -427,12 +458,9 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
       flag_error(err, kErrTimeout);
   } else {
     const int nvec = d / V;
-    for (int i = threadIdx.x; i < NB * nvec; i += kRingWarps * kWarp) {
-      const int b = i / nvec, c = i - b * nvec;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (b < B) v = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)b * d + (size_t)c * V));
-      *reinterpret_cast<uint4 *>(xs + (size_t)b * d + (size_t)c * V) = v;
-    }
+    stage16<8>(reinterpret_cast<uint4 *>(xs), reinterpret_cast<const uint4 *>(x), B * nvec, kRingWarps * kWarp);
+    for (int i = B * nvec + threadIdx.x; i < NB * nvec; i += kRingWarps * kWarp)
+      reinterpret_cast<uint4 *>(xs)[i] = make_uint4(0u, 0u, 0u, 0u);
     named_sync(1, kRingWarps * kWarp);
     bool ok = true;
     for (int i = 0; i < nch; ++i) {
@@ -507,15 +535,38 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
     if (lane == 0 && !ring_produce(W2, r, row0, row1, CR, NSL, NSL, nch, ring, full, empty))
       flag_error(&hdr->err, kErrTimeout);
   } else {
-    for (int i = threadIdx.x; i < NB * r; i += kRingWarps * kWarp) {
-      const int b = i / r, e = i - b * r;
-      const float v = (b < B) ? __ldcg(h + (size_t)b * r + e) : 0.f;
-      int pos = e;
-      if (sizeof(T) == 2) {
-        const int c = e >> 3, q = e & 7;
-        pos = (q < 4) ? (c * 4 + q) : (r / 2 + c * 4 + (q - 4));
+    {
+      // 4 consecutive floats of h land together in one plane (r % 8 == 0 for
+      // fp16, r % 4 == 0 for fp32), so the copy is 16-byte vectors; every
+      // thread issues all its loads before storing
+      constexpr int MAXU = 8;
+      const int n4 = NB * r / 4;
+      const int nt = kRingWarps * kWarp;
+      float4 v[MAXU];
+#pragma unroll
+      for (int u = 0; u < MAXU; ++u) {
+        const int i = threadIdx.x + u * nt;
+        const int b = (i * 4) / r;
+        v[u] = (i < n4 && b < B) ? __ldcg(reinterpret_cast<const float4 *>(h) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      hs[(size_t)b * r + pos] = v;
+      auto place = [&](int i, float4 val) {
+        const int b = (i * 4) / r, e = i * 4 - b * r;
+        int pos = e;
+        if (sizeof(T) == 2) {
+          const int c = e >> 3, q = e & 7;
+          pos = (q < 4) ? (c * 4) : (r / 2 + c * 4);
+        }
+        *reinterpret_cast<float4 *>(hs + (size_t)b * r + pos) = val;
+      };
+#pragma unroll
+      for (int u = 0; u < MAXU; ++u) {
+        const int i = threadIdx.x + u * nt;
+        if (i < n4) place(i, v[u]);
+      }
+      for (int i = threadIdx.x + MAXU * nt; i < n4; i += nt) {
+        const int b = (i * 4) / r;
+        place(i, b < B ? __ldcg(reinterpret_cast<const float4 *>(h) + i) : make_float4(0.f, 0.f, 0.f, 0.f));
+      }
     }
     named_sync(1, kRingWarps * kWarp);
     const int nvec = r / V;
@@ -650,7 +701,7 @@ __global__ void __launch_bounds__(kCompactThreads)
 template <typename T, int NB, int U, bool REGLU>
 __global__ void __launch_bounds__(kThreads)
     k_ffn_gu(const T *__restrict__ Wg, const T *__restrict__ Wu, const float *__restrict__ bias,
-             const T *__restrict__ x, int d, int n, int B, const int32_t *__restrict__ idx,
+             const T *__restrict__ x, int d, long long rs, int n, int B, const int32_t *__restrict__ idx,
              const int32_t *__restrict__ count, float *__restrict__ a, int32_t *__restrict__ err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   T *xs = reinterpret_cast<T *>(smem_raw);
@@ -689,14 +740,14 @@ __global__ void __launch_bounds__(kThreads)
           float ag[NB], au[NB];
 #pragma unroll
           for (int b = 0; b < NB; ++b) ag[b] = au[b] = 0.f;
-          row_dot2<T, NB, U>(Wg + (size_t)k * d, Wu + (size_t)k * d, xs, d, nvec, lane, ag, au);
+          row_dot2<T, NB, U>(Wg + (size_t)k * rs, Wu + (size_t)k * rs, xs, d, nvec, lane, ag, au);
 #pragma unroll
           for (int b = 0; b < NB; ++b) out[b] = fmaxf(warp_sum(ag[b]) + bk, 0.f) * warp_sum(au[b]);
         } else {
           float au[NB];
 #pragma unroll
           for (int b = 0; b < NB; ++b) au[b] = 0.f;
-          row_dot<T, NB, 2 * U>(Wu + (size_t)k * d, xs, d, nvec, lane, au);
+          row_dot<T, NB, 2 * U>(Wu + (size_t)k * rs, xs, d, nvec, lane, au);
 #pragma unroll
           for (int b = 0; b < NB; ++b) out[b] = fmaxf(warp_sum(au[b]) + bk, 0.f);
         }
@@ -717,7 +768,7 @@ __global__ void __launch_bounds__(kThreads)
 template <typename T, int NB, int UJ>
 __global__ void __launch_bounds__(kThreads)
     k_ffn_down(const T *__restrict__ WdT, const float *__restrict__ a, const int32_t *__restrict__ idx,
-               const int32_t *__restrict__ count, int d, int n, int B, int S,
+               const int32_t *__restrict__ count, int d, long long rs, int n, int B, int S,
                float *__restrict__ part, float *__restrict__ y, Header *__restrict__ hdr,
                int prefetch) {
   constexpr int V = Vec<T>::N;
@@ -741,7 +792,7 @@ __global__ void __launch_bounds__(kThreads)
     const uint32_t bytes = (uint32_t)(min(TW, d - col0) * sizeof(T));
     for (int j = js + threadIdx.x; j < je; j += kThreads) {
       const int k = idx ? ld_cg_i32(idx + j) : j;
-      if ((unsigned)k < (unsigned)n) prefetch_l2(WdT + (size_t)k * d + col0, bytes);
+      if ((unsigned)k < (unsigned)n) prefetch_l2(WdT + (size_t)k * rs + col0, bytes);
     }
   }
   pdl_wait();
@@ -762,7 +813,7 @@ __global__ void __launch_bounds__(kThreads)
         int k = -1;
         if (jj < je) k = idx ? ld_cg_i32(idx + jj) : jj;
         const bool ok = (unsigned)k < (unsigned)n;
-        wv[u] = (ok && col_ok) ? ld_stream(WdT + (size_t)k * d + col) : make_uint4(0u, 0u, 0u, 0u);
+        wv[u] = (ok && col_ok) ? ld_stream(WdT + (size_t)k * rs + col) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
         for (int b = 0; b < NB; ++b)
           av[u][b] = (ok && b < nb) ? ld_cg_f32(a + (size_t)jj * B + g0 + b) : 0.f;
@@ -867,7 +918,8 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     k_sparse_ffn(const T *__restrict__ Wg, const T *__restrict__ Wu, const T *__restrict__ WdT,
                  const float *__restrict__ bias, const T *__restrict__ x, int d, int n, int B,
                  const int32_t *__restrict__ idx, const int32_t *__restrict__ count, int NS, int hot_rows,
-                 float *__restrict__ part, float *__restrict__ y, Header *__restrict__ hdr) {
+                 long long rs, int packed, float *__restrict__ part, float *__restrict__ y,
+                 Header *__restrict__ hdr) {
   constexpr int V = Vec<T>::N;
   constexpr int M = REGLU ? 3 : 2;
   constexpr int NW = kFusedWarps;
@@ -899,12 +951,13 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
   // are active for most tokens, so their gate/up/down rows go to L2 while the
   // predictor is still deciding; the bulk copies below then mostly hit L2.
   if (hot_rows > 0 && warp == NW) {
-    const size_t bytes = (size_t)min(hot_rows, n) * d * sizeof(T);
+    // packed layout: the hot rows of all matrices are one contiguous block
+    const size_t rows = (size_t)min(hot_rows, n);
+    const size_t bytes = packed ? rows * (size_t)rs * sizeof(T) : rows * (size_t)d * sizeof(T);
     const size_t per = (bytes / gridDim.x + 15) & ~(size_t)15;
     const size_t o0 = min(bytes, per * blockIdx.x), o1 = min(bytes, o0 + per);
     const T *mats[3] = {REGLU ? Wg : Wu, Wu, WdT};
-#pragma unroll
-    for (int m = REGLU ? 0 : 1; m < 3; ++m) {
+    for (int m = (REGLU || packed) ? 0 : 1; m < (packed ? 1 : 3); ++m) {
       const unsigned char *base = reinterpret_cast<const unsigned char *>(mats[m]);
       for (size_t o = o0 + (size_t)lane * 16384; o < o1; o += 32 * 16384)
         prefetch_l2(base + o, (uint32_t)min((size_t)16384, o1 - o));
@@ -962,13 +1015,15 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
           kslot[s] = k;
           mbar_arrive_expect_tx(&full[s], (uint32_t)M * row_bytes);
           T *dst = stage + (size_t)s * M * d;
-          if constexpr (REGLU) {
-            bulk_g2s(dst, Wg + (size_t)k * d, row_bytes, &full[s]);
-            bulk_g2s(dst + d, Wu + (size_t)k * d, row_bytes, &full[s]);
-            bulk_g2s(dst + 2 * (size_t)d, WdT + (size_t)k * d, row_bytes, &full[s]);
+          if (packed) {          // the neuron's rows are one contiguous block
+            bulk_g2s(dst, (REGLU ? Wg : Wu) + (size_t)k * rs, (uint32_t)M * row_bytes, &full[s]);
+          } else if constexpr (REGLU) {
+            bulk_g2s(dst, Wg + (size_t)k * rs, row_bytes, &full[s]);
+            bulk_g2s(dst + d, Wu + (size_t)k * rs, row_bytes, &full[s]);
+            bulk_g2s(dst + 2 * (size_t)d, WdT + (size_t)k * rs, row_bytes, &full[s]);
           } else {
-            bulk_g2s(dst, Wu + (size_t)k * d, row_bytes, &full[s]);
-            bulk_g2s(dst + d, WdT + (size_t)k * d, row_bytes, &full[s]);
+            bulk_g2s(dst, Wu + (size_t)k * rs, row_bytes, &full[s]);
+            bulk_g2s(dst + d, WdT + (size_t)k * rs, row_bytes, &full[s]);
           }
         }
       }
@@ -976,12 +1031,9 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     }
   } else {
     // ----------------------------------------------------------- consumers --
-    for (int i = threadIdx.x; i < NB * nvec; i += NW * kWarp) {
-      const int b = i / nvec, c = i - b * nvec;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (b < B) v = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)b * d + (size_t)c * V));
-      *reinterpret_cast<uint4 *>(xs + (size_t)b * d + (size_t)c * V) = v;
-    }
+    stage16<8>(reinterpret_cast<uint4 *>(xs), reinterpret_cast<const uint4 *>(x), B * nvec, NW * kWarp);
+    for (int i = B * nvec + threadIdx.x; i < NB * nvec; i += NW * kWarp)
+      reinterpret_cast<uint4 *>(xs)[i] = make_uint4(0u, 0u, 0u, 0u);
     named_sync(1, NW * kWarp);
     // each lane meets the same chunks of x for every neuron: keep them in registers
     uint4 xr[MAXQ][NB];
@@ -1144,7 +1196,7 @@ __global__ void __launch_bounds__(kReduceWarps * kWarp)
 template <typename T, int NB, int U>
 __global__ void __launch_bounds__(kThreads)
     k_act_counts(const T *__restrict__ W, const float *__restrict__ bias, const T *__restrict__ x, int d,
-                 int n, int Ttok, int rpc, int64_t *__restrict__ counts) {
+                 long long rs, int n, int Ttok, int rpc, int64_t *__restrict__ counts) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   T *xs = reinterpret_cast<T *>(smem_raw);
   constexpr int V = Vec<T>::N;
@@ -1168,7 +1220,7 @@ __global__ void __launch_bounds__(kThreads)
         float acc[NB];
 #pragma unroll
         for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-        row_dot<T, NB, U>(W + (size_t)row * d, xs, d, nvec, lane, acc);
+        row_dot<T, NB, U>(W + (size_t)row * rs, xs, d, nvec, lane, acc);
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           const float s = warp_sum(acc[b]) + bk;
@@ -1180,16 +1232,18 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// dst row i = src row perm[i]; one CTA per row (grid-stride), widest copy
-// unit the alignment allows.
+// dst row i (at dst + i*dst_stride) = src row perm[i] (at src + perm[i]*src_stride),
+// row_bytes each; identity when perm is null.  One CTA per row (grid-stride),
+// widest copy unit the alignment allows.
 __global__ void __launch_bounds__(kThreads)
-    k_permute_rows(const unsigned char *__restrict__ src, unsigned char *__restrict__ dst, int n_rows,
-                   long long row_bytes, const int32_t *__restrict__ perm, int unit) {
+    k_permute_rows(const unsigned char *__restrict__ src, long long src_stride, unsigned char *__restrict__ dst,
+                   long long dst_stride, int n_rows, int src_rows, long long row_bytes,
+                   const int32_t *__restrict__ perm, int unit) {
   for (int i = blockIdx.x; i < n_rows; i += gridDim.x) {
-    const int p = __ldg(perm + i);
-    if ((unsigned)p >= (unsigned)n_rows) continue;
-    const unsigned char *s = src + (size_t)p * row_bytes;
-    unsigned char *t = dst + (size_t)i * row_bytes;
+    const int p = perm ? __ldg(perm + i) : i;
+    if ((unsigned)p >= (unsigned)src_rows) continue;
+    const unsigned char *s = src + (size_t)p * src_stride;
+    unsigned char *t = dst + (size_t)i * dst_stride;
     if (unit == 16) {
       for (long long o = threadIdx.x; o < row_bytes / 16; o += blockDim.x)
         reinterpret_cast<uint4 *>(t)[o] = __ldg(reinterpret_cast<const uint4 *>(s) + o);
@@ -1287,6 +1341,20 @@ int down_splits(const asf_ffn *f) {
 size_t mask_region(const asf_predictor *p) {
   return r256((size_t)std::max(n_words_of(p->n), kMaxGrid) * 4);
 }
+// Row stride of the FFN matrices in elements (0 in the descriptor = d).
+long long ffn_rs(const asf_ffn *f) { return f->row_stride > 0 ? (long long)f->row_stride : (long long)f->d; }
+
+// Neuron-major packed layout: a neuron's gate/up/down rows are one contiguous
+// block of M*d elements, so one bulk copy fetches all of them.
+bool ffn_packed(const asf_ffn *f) {
+  const int M = f->act == ASF_ACT_REGLU ? 3 : 2;
+  const size_t rb = (size_t)f->d * esize(f->wdtype);
+  if (ffn_rs(f) != (long long)M * f->d) return false;
+  const char *first = static_cast<const char *>(f->act == ASF_ACT_REGLU ? f->Wg : f->Wu);
+  if (f->act == ASF_ACT_REGLU && static_cast<const char *>(f->Wu) != first + rb) return false;
+  return static_cast<const char *>(f->WdT) == first + (size_t)(M - 1) * rb;
+}
+
 size_t pred_scratch(const asf_predictor *p, int B) { return mask_region(p) + r256((size_t)B * p->r * 4); }
 size_t ffn_scratch(const asf_ffn *f, int B) {
   const size_t two_kernel = r256((size_t)f->n * B * 4) + r256((size_t)down_splits(f) * B * f->d * 4);
@@ -1313,6 +1381,9 @@ asf_status check_ffn(const asf_ffn *f) {
   if (f->act == ASF_ACT_REGLU && !f->Wg) return ASF_ERR_INVALID_ARG;
   if (f->d <= 0 || f->n <= 0) return ASF_ERR_INVALID_ARG;
   if (f->d % vec_of(f->wdtype)) return ASF_ERR_MISALIGNED;
+  if (f->row_stride < 0 || (f->row_stride > 0 && f->row_stride < f->d)) return ASF_ERR_INVALID_ARG;
+  if (f->row_stride % vec_of(f->wdtype)) return ASF_ERR_MISALIGNED;
+  if (f->hot_rows < 0) return ASF_ERR_INVALID_ARG;
   if ((size_t)f->d * esize(f->wdtype) > kSmemBudget) return ASF_ERR_UNSUPPORTED;
   if (down_tiles(f) > kMaxTiles) return ASF_ERR_UNSUPPORTED;
   if (!al16(f->Wu) || !al16(f->WdT) || (f->Wg && !al16(f->Wg)) || !al4(f->bias)) return ASF_ERR_MISALIGNED;
@@ -1358,8 +1429,15 @@ cudaError_t run_pred_l2(const asf_predictor *p, int B, float thr, const float *h
 }
 
 constexpr size_t kRingChunk = 32 * 1024;    // bytes per bulk copy of a ring slot
-constexpr size_t kRing1Smem = 80 * 1024;     // layer-1 ring + x: fits beside the fused FFN
-constexpr size_t kRing2Smem = 168 * 1024;
+constexpr size_t kRing1Smem = 80 * 1024;     // layer-1 ring + x
+size_t ring2_budget() {
+  static size_t kb = (size_t)env_flag("ASFFN_RING2_KB", 168);
+  return std::min<size_t>(std::max<size_t>(kb, 40), 200) * 1024;
+}
+bool ring1_enabled() {
+  static int on = env_flag("ASFFN_RING1", 1);
+  return on != 0;
+}
 
 // rows per chunk and slots for a ring over rows of row_bytes within budget
 bool ring_shape(size_t row_bytes, size_t vec_bytes, size_t budget, int rpc, int &CR, int &NSL) {
@@ -1394,7 +1472,7 @@ cudaError_t run_pred2_ring(const asf_predictor *p, int B, float thr, const float
   const int grid = (p->n + rpc - 1) / rpc;
   const size_t vec = (size_t)NB * p->r * 4 + ((size_t)rpc / 32 + 2) * 4;
   int CR, NSL;
-  used = ring_shape((size_t)p->r * sizeof(T), vec, kRing2Smem, rpc, CR, NSL);
+  used = ring_shape((size_t)p->r * sizeof(T), vec, ring2_budget(), rpc, CR, NSL);
   if (!used) return cudaSuccess;
   const size_t smem = ring_layout(NSL, CR, p->r, (int)sizeof(T), vec).total;
   (void)idx;
@@ -1467,7 +1545,7 @@ asf_status predict_t(const asf_predictor *p, const void *x, int B, float thr, in
   const bool ring = B <= 8 && ring_enabled() && n_words_of(p->n) <= kCompactThreads * kCompactWords;
   bool used = false;
   cudaError_t e = cudaSuccess;
-  if (ring) e = pred1_ring_any<T>(p, x, B, h, mask, &hdr->err, st, used);
+  if (ring && ring1_enabled()) e = pred1_ring_any<T>(p, x, B, h, mask, &hdr->err, st, used);
   if (e == cudaSuccess && !used) e = pred1_reg_any<T>(p, x, B, h, mask, st);
   if (e != cudaSuccess) return ASF_ERR_CUDA;
   used = false;
@@ -1487,9 +1565,9 @@ cudaError_t run_gu(const asf_ffn *f, const void *x, int B, const int32_t *idx, c
   const size_t smem = (size_t)NB * f->d * sizeof(T);
   if (f->act == ASF_ACT_REGLU)
     return launch(k_ffn_gu<T, NB, (NB <= 2 ? 8 : 4), true>, dim3(grid), dim3(kThreads), smem, st, (const T *)f->Wg,
-                  (const T *)f->Wu, f->bias, (const T *)x, f->d, f->n, B, idx, count, a, err);
+                  (const T *)f->Wu, f->bias, (const T *)x, f->d, ffn_rs(f), f->n, B, idx, count, a, err);
   return launch(k_ffn_gu<T, NB, (NB <= 2 ? 8 : 4), false>, dim3(grid), dim3(kThreads), smem, st, (const T *)f->Wg,
-                (const T *)f->Wu, f->bias, (const T *)x, f->d, f->n, B, idx, count, a, err);
+                (const T *)f->Wu, f->bias, (const T *)x, f->d, ffn_rs(f), f->n, B, idx, count, a, err);
 }
 
 template <typename T, int NB>
@@ -1500,7 +1578,7 @@ cudaError_t run_down(const asf_ffn *f, int B, const int32_t *idx, const int32_t 
   const int S = down_splits(f);
   const size_t smem = (size_t)kWarps * NB * TW * 4;
   return launch(k_ffn_down<T, NB, 4>, dim3(ct, S), dim3(kThreads), smem, st, (const T *)f->WdT, a, idx, count,
-                f->d, f->n, B, S, part, y, hdr, prefetch_enabled());
+                f->d, ffn_rs(f), f->n, B, S, part, y, hdr, prefetch_enabled());
 }
 
 // ------------------------------------------------------------- fused ffn --
@@ -1543,7 +1621,7 @@ cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *i
     const int G = fused_grid();
     cudaError_t e = launch(kern, dim3(G), dim3(threads), L.total, st, (const T *)f->Wg, (const T *)f->Wu,
                            (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count, NS,
-                           idx ? std::max(0, f->hot_rows) : 0, part, y, hdr);
+                           idx ? std::max(0, f->hot_rows) : 0, ffn_rs(f), ffn_packed(f) ? 1 : 0, part, y, hdr);
     if (e != cudaSuccess) return e;
     return launch(k_reduce_partials, dim3((f->d + kWarp - 1) / kWarp, B), dim3(kReduceWarps * kWarp), 0, st,
                   (const float *)part, G, B, f->d, y);
@@ -1618,10 +1696,10 @@ asf_status counts_t(const asf_ffn *f, const void *x, int Ttok, int64_t *counts, 
   const size_t smem = (size_t)nb * f->d * sizeof(T);
   cudaError_t e;
   switch (nb) {
-    case 1: e = launch(k_act_counts<T, 1, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, f->n, Ttok, rpc, counts); break;
-    case 2: e = launch(k_act_counts<T, 2, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, f->n, Ttok, rpc, counts); break;
-    case 4: e = launch(k_act_counts<T, 4, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, f->n, Ttok, rpc, counts); break;
-    default: e = launch(k_act_counts<T, 8, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, f->n, Ttok, rpc, counts); break;
+    case 1: e = launch(k_act_counts<T, 1, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, ffn_rs(f), f->n, Ttok, rpc, counts); break;
+    case 2: e = launch(k_act_counts<T, 2, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, ffn_rs(f), f->n, Ttok, rpc, counts); break;
+    case 4: e = launch(k_act_counts<T, 4, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, ffn_rs(f), f->n, Ttok, rpc, counts); break;
+    default: e = launch(k_act_counts<T, 8, 4>, dim3(grid), dim3(kThreads), smem, st, (const T *)W, f->bias, (const T *)x, f->d, ffn_rs(f), f->n, Ttok, rpc, counts); break;
   }
   return cuda_status(e);
 }
@@ -1659,7 +1737,7 @@ asf_status noalloc_scratch(void **out) {
 // ======================================================================== //
 extern "C" {
 
-int32_t asf_version(void) { return 101; }
+int32_t asf_version(void) { return 102; }
 
 const char *asf_status_string(asf_status s) {
   switch (s) {
@@ -1774,8 +1852,33 @@ asf_status asf_permute_rows(const void *src, void *dst, int32_t n_rows, int64_t 
     unit = 4;
   const int grid = std::min(n_rows, 8 * sm_count());
   return cuda_status(launch(k_permute_rows, dim3(grid), dim3(kThreads), 0, (cudaStream_t)stream,
-                            (const unsigned char *)src, (unsigned char *)dst, (int)n_rows, (long long)row_bytes,
-                            perm, unit));
+                            (const unsigned char *)src, (long long)row_bytes, (unsigned char *)dst,
+                            (long long)row_bytes, (int)n_rows, (int)n_rows, (long long)row_bytes, perm, unit));
+}
+
+asf_status asf_gather_rows(const void *src, int64_t src_stride, int32_t src_rows, void *dst, int64_t dst_stride,
+                           int32_t n_rows, int64_t row_bytes, const int32_t *perm, asf_stream_t stream) {
+  if (!src || !dst || n_rows < 0 || src_rows < 0 || row_bytes <= 0) return ASF_ERR_INVALID_ARG;
+  if (src_stride < row_bytes || dst_stride < row_bytes) return ASF_ERR_INVALID_ARG;
+  if (!perm && n_rows > src_rows) return ASF_ERR_INVALID_ARG;
+  if (perm && !al4(perm)) return ASF_ERR_MISALIGNED;
+  // the source and destination row ranges must not overlap
+  const char *s0 = static_cast<const char *>(src), *d0 = static_cast<const char *>(dst);
+  const char *s1 = s0 + (size_t)(src_rows > 0 ? src_rows - 1 : 0) * src_stride + row_bytes;
+  const char *d1 = d0 + (size_t)(n_rows > 0 ? n_rows - 1 : 0) * dst_stride + row_bytes;
+  if (n_rows > 0 && src_rows > 0 && s0 < d1 && d0 < s1) return ASF_ERR_INVALID_ARG;
+  if (n_rows == 0) return ASF_OK;
+  int unit = 1;
+  const auto a16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  const auto a4 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
+  if (row_bytes % 16 == 0 && src_stride % 16 == 0 && dst_stride % 16 == 0 && a16(src) && a16(dst))
+    unit = 16;
+  else if (row_bytes % 4 == 0 && src_stride % 4 == 0 && dst_stride % 4 == 0 && a4(src) && a4(dst))
+    unit = 4;
+  const int grid = std::min(n_rows, 8 * sm_count());
+  return cuda_status(launch(k_permute_rows, dim3(grid), dim3(kThreads), 0, (cudaStream_t)stream,
+                            (const unsigned char *)src, (long long)src_stride, (unsigned char *)dst,
+                            (long long)dst_stride, (int)n_rows, (int)src_rows, (long long)row_bytes, perm, unit));
 }
 
 asf_status asf_sparse_ffn_noalloc(const asf_ffn *ffn, const void *x, int32_t B, const int32_t *idx,

@@ -43,6 +43,8 @@ def parse_args(argv=None):
     p.add_argument("--batch", type=int, default=1)
     p.add_argument("--mode", choices=["predict", "sparse", "dense"], default="predict")
     p.add_argument("--no-hot-perm", action="store_true", help="keep neuron id order")
+    p.add_argument("--layout", choices=["packed", "split"], default="packed",
+                   help="FFN weight layout: neuron-major packed rows, or separate W_gate/W_up/W_down^T")
     p.add_argument("--no-hot-prefetch", action="store_true",
                    help="do not pass the hot-row prefetch hint to the sparse FFN")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -237,7 +239,7 @@ def workload_config(cfg, args):
     return {"workload": (f"{cfg.name}: {cfg.layers} layers, d={cfg.d}, d_ffn={cfg.n}, predictor "
                          f"{cfg.d}->{cfg.r}->{cfg.n}, {cfg.act}, {cfg.dtype} weights, batch {args.batch}, "
                          f"Zipf({cfg.gamma}) with {cfg.frac:.0%} mean activity, tau={cfg.tau}, "
-                         f"hot rows {'first' if hot else 'in id order'}, mode {args.mode}"),
+                         f"hot rows {'first' if hot else 'in id order'}, {args.layout} layout, mode {args.mode}"),
             "layers": cfg.layers, "batch": args.batch,
             "tokens_cycled": args.tokens if args.tokens > 0 else cfg.tokens,
             "weights": cfg.dtype, "accumulate": "f32",
@@ -273,6 +275,7 @@ def hot_permute_layer(cfg, layer, w, device):
     new = type(w)(w.act, w.dtype, prow(w.Wg), prow(w.Wu), prow(w.WdT), prow(w.bias), w.W1, w.b1,
                   prow(w.W2), prow(w.b2), w.p[perm])
     torch.cuda.synchronize()
+    del w
     k_hot = int(cfg.n * cfg.hot_ratio)
     share = float(c[perm[:k_hot]].sum()) / max(1, int(c.sum()))
     # leading rows active for at least half of the calibration tokens: the
@@ -321,7 +324,19 @@ def run_ours(args, cfg):
             shares.append(share)
             hot_rows.append(0 if args.no_hot_prefetch else hr)
         weights.append(w)
-    preds, ffns = build_layers(weights, device, hot_rows if hot else None)
+    if args.layout == "packed":
+        # neuron-major packed rows: one bulk copy per neuron in the sparse FFN
+        from activation_sparse_ffn_predict_b200.api import FFN, Predictor, pack_layer
+        preds, ffns = [], []
+        for l, w in enumerate(weights):
+            pk = pack_layer(w.act, w.Wg, w.Wu, w.WdT)
+            preds.append(Predictor(w.W1, w.b1, w.W2, w.b2))
+            ffns.append(FFN.packed(w.act, pk, w.bias, hot_rows=(hot_rows[l] if hot else 0)))
+            w.Wg = w.Wu = w.WdT = None      # the packed copy replaces the split matrices
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    else:
+        preds, ffns = build_layers(weights, device, hot_rows if hot else None)
     st = LayerStack(preds, ffns, B, cfg.tau, mode=args.mode, device=device)
     # token stream: each rank decodes its own tokens (replicas; no collectives)
     X = torch.empty(T, L, B, cfg.d, dtype=st.dtype, device=device)

@@ -97,6 +97,11 @@ typedef struct {
                          first by the offline permutation); asf_sparse_ffn prefetches them
                          into L2 while the list is still being predicted.  0 = no hint.
                          Affects speed only, never results. */
+  int32_t row_stride; /* elements between consecutive rows of Wg/Wu/WdT; 0 means d.  With
+                         row_stride = m*d and Wu = Wg + d, WdT = Wu + d (REGLU; for RELU
+                         WdT = Wu + d) the layer is in the neuron-major packed layout
+                         (gate|up|down of a neuron contiguous, see asf_gather_rows), and the
+                         sparse FFN fetches each neuron with one bulk copy. */
 } asf_ffn;
 
 /* Bytes of device workspace needed by asf_predict / asf_sparse_ffn /
@@ -144,6 +149,16 @@ ASF_API asf_status asf_dense_ffn(const asf_ffn *ffn, const void *x, int32_t B, f
 ASF_API asf_status asf_activation_counts(const asf_ffn *ffn, const void *x, int32_t T, int64_t *counts,
                                  void *ws, size_t ws_bytes, asf_stream_t stream);
 
+/* Strided row gather on the device: dst row i (at dst + i*dst_stride bytes) =
+ * src row p (at src + p*src_stride bytes) with p = perm[i] (p = i when perm is
+ * NULL), row_bytes each, for i < n_rows; rows with p outside [0, src_rows) are
+ * skipped.  With dst_stride = m*d*s and dst offsets 0, d*s, 2*d*s it builds the
+ * neuron-major packed layout of asf_ffn (and applies a hot permutation in the
+ * same pass).  Source and destination ranges must not overlap. */
+ASF_API asf_status asf_gather_rows(const void *src, int64_t src_stride, int32_t src_rows, void *dst,
+                                   int64_t dst_stride, int32_t n_rows, int64_t row_bytes,
+                                   const int32_t *perm, asf_stream_t stream);
+
 /* Host-side, synchronous: perm = neuron ids in descending count order, equal
  * counts in ascending id order.  counts: host int64 [n]; perm_out: host int32 [n]. */
 ASF_API asf_status asf_hot_permutation(const int64_t *counts, int32_t n, int32_t *perm_out);
@@ -188,7 +203,7 @@ ASF_API asf_status asf_read_error(void *ws, int32_t *host_out, asf_stream_t stre
 /* Static description of a status code. */
 ASF_API const char *asf_status_string(asf_status s);
 
-/* ABI version: major * 100 + minor (1.01 added asf_ffn.hot_rows). */
+/* ABI version: major * 100 + minor (1.02: asf_ffn.hot_rows, asf_ffn.row_stride, asf_gather_rows). */
 ASF_API int32_t asf_version(void);
 
 #ifdef __cplusplus

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.asf_version() == 101
+    assert lib.asf_version() == 102
     for code in range(8):
         assert lib.asf_status_string(code).decode() not in ("", "unknown status")
     assert lib.asf_status_string(99).decode() == "unknown status"
@@ -58,7 +58,7 @@ def test_struct_layout_matches_header():
     # int32 d, r, n; enum; then four pointers (8-byte aligned)
     assert ctypes.sizeof(L.asf_predictor) == 16 + 4 * 8
     assert L.asf_predictor.W1.offset == 16
-    assert ctypes.sizeof(L.asf_ffn) == 16 + 4 * 8 + 8   # + hot_rows (padded)
+    assert ctypes.sizeof(L.asf_ffn) == 16 + 4 * 8 + 8   # + hot_rows, row_stride
     assert L.asf_ffn.Wg.offset == 16
 
 

@@ -253,3 +253,51 @@ def test_hot_row_hint_changes_nothing_but_speed(layer):
         torch.cuda.synchronize()
         assert torch.equal(y0, y1)
     assert layer.error() == 0
+
+
+def test_packed_layout_is_bitwise_equal_to_split_layout(layer):
+    # Neuron-major packed rows (one bulk copy per neuron) change the memory
+    # layout only: every FFN path must give bit-identical results.
+    cfg = layer.cfg
+    w = layer.w
+    packed = A.pack_layer(w.act, w.Wg, w.Wu, w.WdT)
+    pf = A.FFN.packed(w.act, packed, w.bias, hot_rows=cfg.n // 4)
+    for B in (1, 4, 16):
+        rows = slice(0, B)
+        x = layer.Xd[rows].contiguous()
+        ids = layer.oracle_idx(rows)
+        idt = torch.zeros(cfg.n, dtype=torch.int32, device="cuda")
+        if ids.size:
+            idt[:ids.size] = torch.from_numpy(ids).cuda()
+        cnt = torch.tensor([ids.size], dtype=torch.int32, device="cuda")
+        ys = torch.zeros(B, cfg.d, dtype=torch.float32, device="cuda")
+        yp = torch.zeros(B, cfg.d, dtype=torch.float32, device="cuda")
+        A.asf_sparse_ffn(layer.ffn, x, idt, cnt, ys, layer.ws)
+        A.asf_sparse_ffn(pf, x, idt, cnt, yp, layer.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(ys, yp), B
+        A.asf_dense_ffn(layer.ffn, x, ys, layer.ws)
+        A.asf_dense_ffn(pf, x, yp, layer.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(ys, yp), B
+    Xc = S.layer_tokens(cfg, 0, 64, kind="x_calib").cuda().contiguous()
+    c1 = torch.zeros(cfg.n, dtype=torch.int64, device="cuda")
+    c2 = torch.zeros(cfg.n, dtype=torch.int64, device="cuda")
+    A.asf_activation_counts(layer.ffn, Xc, c1, layer.ws)
+    A.asf_activation_counts(pf, Xc, c2, layer.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2)
+    assert layer.error() == 0
+
+
+def test_gather_rows_strided_and_permuted():
+    ensure_built()
+    src = torch.arange(9 * 24, dtype=torch.int16, device="cuda").reshape(9, 24)
+    perm = torch.tensor([8, 0, 3, 3, 7, 1, 2, 6, 5], dtype=torch.int32, device="cuda")
+    dst = torch.full((9, 2, 24), -1, dtype=torch.int16, device="cuda")
+    A.asf_gather_rows(src, dst, perm, dst_offset=48, dst_stride=96)
+    torch.cuda.synchronize()
+    assert torch.equal(dst[:, 1].cpu(), src.cpu()[perm.cpu().long()])
+    assert (dst[:, 0] == -1).all()
+    with pytest.raises(ValueError):
+        A.asf_gather_rows(src, dst, perm, dst_offset=96, dst_stride=96)

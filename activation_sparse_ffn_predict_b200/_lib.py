@@ -32,7 +32,8 @@ class asf_predictor(ctypes.Structure):
 class asf_ffn(ctypes.Structure):
     _fields_ = [("d", c_int32), ("n", c_int32), ("wdtype", c_int), ("act", c_int),
                 ("Wg", c_void_p), ("Wu", c_void_p), ("WdT", c_void_p), ("bias", c_void_p),
-                ("hot_rows", c_int32), ("row_stride", c_int32)]
+                ("hot_rows", c_int32), ("row_stride", c_int32),
+                ("l2_next", c_void_p * 2), ("l2_next_bytes", ctypes.c_int64 * 2)]
 
 
 # name -> (restype, argtypes), exactly the declarations of include/asffn.h

@@ -101,6 +101,19 @@ class FFN:
         self.desc = L.asf_ffn(d, n, _DT[Wu.dtype], _ACT[act], gp, _dev(Wu, "Wu"), _dev(WdT, "WdT"),
                               _dev(bias, "bias", torch.float32), self.hot_rows, 0)
 
+    def set_l2_next(self, *ranges: torch.Tensor) -> "FFN":
+        """L2 prefetch hint (asf_ffn.l2_next): up to two contiguous device
+        tensors that are read soon after each sparse-FFN call on this layer,
+        typically the next layer's predictor weights.  No argument clears it."""
+        if len(ranges) > 2:
+            raise ValueError("at most two ranges")
+        ptrs = [_dev(t, "l2_next") for t in ranges]
+        self.l2_next = tuple(ranges)          # keeps the memory alive
+        for i in range(2):
+            self.desc.l2_next[i] = ptrs[i].value if i < len(ptrs) else None
+            self.desc.l2_next_bytes[i] = ranges[i].numel() * ranges[i].element_size() if i < len(ranges) else 0
+        return self
+
 
 def asf_version() -> int:
     return int(L.load().asf_version())

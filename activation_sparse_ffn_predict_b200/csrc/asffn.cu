@@ -149,6 +149,27 @@ __device__ __forceinline__ void prefetch_range(const void *p, size_t bytes) {
     prefetch_l2(c + o, (uint32_t)min(kPiece, bytes - o));
 }
 
+// Up to two device ranges to pull into L2 for whatever runs next (the
+// asf_ffn.l2_next hint).  Sizes are multiples of 16 bytes.
+struct L2Next {
+  const unsigned char *p[2];
+  long long bytes[2];
+};
+
+// Lanes of one warp issue this CTA's share (part of parts) of the ranges in
+// 32 KB pieces, piece q going to part q mod parts.
+__device__ __forceinline__ void prefetch_next(const L2Next &nx, int part, int parts) {
+  constexpr long long kPiece = 32768;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if (!nx.p[i]) continue;
+    const long long np = (nx.bytes[i] + kPiece - 1) / kPiece;
+    for (long long q = part + (long long)parts * lane; q < np; q += (long long)parts * kWarp)
+      prefetch_l2(nx.p[i] + q * kPiece, (uint32_t)min(kPiece, nx.bytes[i] - q * kPiece));
+  }
+}
+
 // Copy n16 16-byte units from global (data written by the previous kernel,
 // read through L2) into shared memory using the first `nthreads` threads.  All
 // of a thread's loads are issued before its first store, so the copy costs one
@@ -211,8 +232,8 @@ __global__ void __launch_bounds__(kThreads)
       float acc[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+      const float bias = __ldg(b1 + row);     // in flight with the row's loads
       row_dot<T, NB, U>(W1 + (size_t)row * d, xs, d, nvec, lane, acc);
-      const float bias = __ldg(b1 + row);
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         const float s = warp_sum(acc[b]);
@@ -282,10 +303,13 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
     for (int rb = row0 + warp * R; rb < row1; rb += kWarps * R) {
       float acc[R][NB];
+      float bq[R];     // in flight with the rows' loads
 #pragma unroll
-      for (int q = 0; q < R; ++q)
+      for (int q = 0; q < R; ++q) {
+        bq[q] = (rb + q < row1) ? __ldg(b2 + rb + q) : 0.f;
 #pragma unroll
         for (int b = 0; b < NB; ++b) acc[q][b] = 0.f;
+      }
       for (int c0 = lane; c0 < nvec; c0 += UC * kWarp) {
         uint4 wv[R][UC];
 #pragma unroll
@@ -312,7 +336,7 @@ __global__ void __launch_bounds__(kThreads)
       for (int q = 0; q < R; ++q) {
         const int row = rb + q;
         bool on = false;
-        const float bias = (row < row1) ? __ldg(b2 + row) : 0.f;
+        const float bias = bq[q];
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           const float z = warp_sum(acc[q][b]) + bias;
@@ -494,6 +518,12 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
   }
 }
 
+// Shared bytes of k_pred2_ring besides the ring: staged h [NB][r], the CTA's
+// mask words, and its b2 values.
+__host__ __device__ inline size_t pred2_vec_bytes(int NB, int r, int rpc) {
+  return (size_t)NB * r * 4 + (size_t)(rpc / 32 + 2) * 4 + (size_t)rpc * 4;
+}
+
 // Layer 2 + threshold + union over tokens, B <= NB tokens, with W2 rows fed by
 // the bulk-copy ring (first chunks issued before the wait).  Each CTA ORs the
 // bits of its rows into the union mask; the next kernel compacts it.
@@ -506,11 +536,12 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
   constexpr int V = Vec<T>::N;
   constexpr int NT = (kRingWarps + 1) * kWarp;
   const int nwl_max = rpc / 32 + 2;
-  const RingLayout L = ring_layout(NSL, CR, r, (int)sizeof(T), (size_t)NB * r * 4 + (size_t)nwl_max * 4);
+  const RingLayout L = ring_layout(NSL, CR, r, (int)sizeof(T), pred2_vec_bytes(NB, r, rpc));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
   uint64_t *empty = reinterpret_cast<uint64_t *>(smem + L.empty);
   float *hs = reinterpret_cast<float *>(smem + L.vec);
   uint32_t *smask = reinterpret_cast<uint32_t *>(smem + L.vec + (size_t)NB * r * 4);
+  float *sb = reinterpret_cast<float *>(smask + nwl_max);     // b2 of this CTA's rows
   T *ring = reinterpret_cast<T *>(smem + L.ring);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = blockIdx.x * rpc, row1 = min(n, row0 + rpc);
@@ -529,6 +560,10 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
   if (warp == kRingWarps && lane == 0) {
     for (int i = 0; i < min(nch, NSL); ++i) ring_issue(W2, r, row0, row1, CR, NSL, i, ring, full);
   }
+  // biases are weights too: fetched before the wait, read from shared memory
+  // (the consumers' named barrier below orders these stores)
+  if (warp < kRingWarps)
+    for (int i = threadIdx.x; i < row1 - row0; i += kRingWarps * kWarp) sb[i] = __ldg(b2 + row0 + i);
   pdl_trigger();
   pdl_wait();
   if (warp == kRingWarps) {
@@ -626,7 +661,7 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
           }
         }
         bool on = false;
-        const float bias = __ldg(b2 + row);
+        const float bias = sb[row - row0];
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           const float z = warp_sum(acc[b]) + bias;
@@ -770,7 +805,7 @@ __global__ void __launch_bounds__(kThreads)
     k_ffn_down(const T *__restrict__ WdT, const float *__restrict__ a, const int32_t *__restrict__ idx,
                const int32_t *__restrict__ count, int d, long long rs, int n, int B, int S,
                float *__restrict__ part, float *__restrict__ y, Header *__restrict__ hdr,
-               int prefetch) {
+               int prefetch, L2Next nx) {
   constexpr int V = Vec<T>::N;
   constexpr int TW = kWarp * V;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -795,6 +830,7 @@ __global__ void __launch_bounds__(kThreads)
       if ((unsigned)k < (unsigned)n) prefetch_l2(WdT + (size_t)k * rs + col0, bytes);
     }
   }
+  if (warp == kWarps - 1) prefetch_next(nx, blockIdx.y * gridDim.x + blockIdx.x, gridDim.x * gridDim.y);
   pdl_wait();
   pdl_trigger();
   for (int g0 = 0; g0 < B; g0 += NB) {
@@ -877,10 +913,11 @@ __global__ void __launch_bounds__(kThreads)
 // Shared-memory layout of k_sparse_ffn for NS ring slots of M rows of d elements.
 struct FusedLayout {
   int NS, grp;
-  size_t full, empty, kslot, pd, x, stage, red, total;
+  size_t full, empty, kslot, bias, pd, x, stage, red, total;
 };
 
-__host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int esz, int NB) {
+// nl_max: most list positions one CTA takes (ceil(n / grid)).
+__host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int esz, int NB, int nl_max) {
   FusedLayout L;
   L.NS = NS;
   L.grp = NS / 2 > 0 ? NS / 2 : 1;
@@ -888,6 +925,7 @@ __host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int es
   L.full = o;  o += (size_t)NS * 8;
   L.empty = o; o += (size_t)NS * 8;
   L.kslot = o; o += (size_t)NS * 4;
+  L.bias = o;  o += (size_t)nl_max * 4;
   o = align_up(o, 16);
   L.pd = o;    o += (size_t)kFusedWarps * L.grp * 2 * NB * 4;
   o = align_up(o, 128);
@@ -925,10 +963,11 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
   constexpr int NW = kFusedWarps;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_fail;
-  const FusedLayout L = fused_layout(NS, d, M, (int)sizeof(T), NB);
+  const FusedLayout L = fused_layout(NS, d, M, (int)sizeof(T), NB, (n + (int)gridDim.x - 1) / (int)gridDim.x);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
   uint64_t *empty = reinterpret_cast<uint64_t *>(smem + L.empty);
   int *kslot = reinterpret_cast<int *>(smem + L.kslot);
+  float *sbias = reinterpret_cast<float *>(smem + L.bias);    // bias of list position js + i
   float *pd = reinterpret_cast<float *>(smem + L.pd);
   T *xs = reinterpret_cast<T *>(smem + L.x);
   T *stage = reinterpret_cast<T *>(smem + L.stage);
@@ -1034,6 +1073,11 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     stage16<8>(reinterpret_cast<uint4 *>(xs), reinterpret_cast<const uint4 *>(x), B * nvec, NW * kWarp);
     for (int i = B * nvec + threadIdx.x; i < NB * nvec; i += NW * kWarp)
       reinterpret_cast<uint4 *>(xs)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // the biases of this CTA's neurons, while the first rows are in flight
+    for (int i = threadIdx.x; i < nl; i += NW * kWarp) {
+      const int k = idx ? ld_cg_i32(idx + js + i) : js + i;
+      sbias[i] = (unsigned)k < (unsigned)n ? __ldg(bias + k) : 0.f;
+    }
     named_sync(1, NW * kWarp);
     // each lane meets the same chunks of x for every neuron: keep them in registers
     uint4 xr[MAXQ][NB];
@@ -1103,7 +1147,7 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
           }
           float v = 0.f;
           if (k >= 0 && b < B) {
-            const float bk = __ldg(bias + k);
+            const float bk = sbias[i];
             v = REGLU ? fmaxf(g + bk, 0.f) * u : fmaxf(u + bk, 0.f);
           }
           a[b] = v;
@@ -1159,9 +1203,12 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
 constexpr int kReduceWarps = 8;
 constexpr int kReduceMaxPerWarp = 32;   // G <= 256
 __global__ void __launch_bounds__(kReduceWarps * kWarp)
-    k_reduce_partials(const float *__restrict__ part, int G, int B, int d, float *__restrict__ y) {
+    k_reduce_partials(const float *__restrict__ part, int G, int B, int d, float *__restrict__ y, L2Next nx) {
   __shared__ float red[kReduceWarps][kWarp];
   pdl_trigger();
+  // This grid starts while the sparse FFN still streams its rows; the hinted
+  // ranges fill L2 in that time.
+  if (threadIdx.x < kWarp) prefetch_next(nx, blockIdx.y * gridDim.x + blockIdx.x, gridDim.x * gridDim.y);
   pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int col = blockIdx.x * kWarp + lane;
@@ -1374,6 +1421,16 @@ asf_status check_pred(const asf_predictor *p) {
   return ASF_OK;
 }
 
+L2Next l2_next_of(const asf_ffn *f) {
+  L2Next nx{};
+  for (int i = 0; i < 2; ++i) {
+    const long long b = f->l2_next[i] ? (f->l2_next_bytes[i] & ~15ll) : 0;
+    nx.p[i] = b > 0 ? static_cast<const unsigned char *>(f->l2_next[i]) : nullptr;
+    nx.bytes[i] = b > 0 ? b : 0;
+  }
+  return nx;
+}
+
 asf_status check_ffn(const asf_ffn *f) {
   if (!f || !f->Wu || !f->WdT || !f->bias) return ASF_ERR_INVALID_ARG;
   if (f->wdtype != ASF_F16 && f->wdtype != ASF_F32) return ASF_ERR_UNSUPPORTED;
@@ -1384,6 +1441,10 @@ asf_status check_ffn(const asf_ffn *f) {
   if (f->row_stride < 0 || (f->row_stride > 0 && f->row_stride < f->d)) return ASF_ERR_INVALID_ARG;
   if (f->row_stride % vec_of(f->wdtype)) return ASF_ERR_MISALIGNED;
   if (f->hot_rows < 0) return ASF_ERR_INVALID_ARG;
+  for (int i = 0; i < 2; ++i) {
+    if (f->l2_next_bytes[i] < 0) return ASF_ERR_INVALID_ARG;
+    if (f->l2_next[i] && !al16(f->l2_next[i])) return ASF_ERR_MISALIGNED;
+  }
   if ((size_t)f->d * esize(f->wdtype) > kSmemBudget) return ASF_ERR_UNSUPPORTED;
   if (down_tiles(f) > kMaxTiles) return ASF_ERR_UNSUPPORTED;
   if (!al16(f->Wu) || !al16(f->WdT) || (f->Wg && !al16(f->Wg)) || !al4(f->bias)) return ASF_ERR_MISALIGNED;
@@ -1431,11 +1492,11 @@ cudaError_t run_pred_l2(const asf_predictor *p, int B, float thr, const float *h
 constexpr size_t kRingChunk = 32 * 1024;    // bytes per bulk copy of a ring slot
 constexpr size_t kRing1Smem = 80 * 1024;     // layer-1 ring + x
 size_t ring2_budget() {
-  static size_t kb = (size_t)env_flag("ASFFN_RING2_KB", 168);
+  static size_t kb = (size_t)env_flag("ASFFN_RING2_KB", 136);
   return std::min<size_t>(std::max<size_t>(kb, 40), 200) * 1024;
 }
 bool ring1_enabled() {
-  static int on = env_flag("ASFFN_RING1", 1);
+  static int on = env_flag("ASFFN_RING1", 0);
   return on != 0;
 }
 
@@ -1470,7 +1531,7 @@ cudaError_t run_pred2_ring(const asf_predictor *p, int B, float thr, const float
   const int sms = sm_count();
   const int rpc = (p->n + sms - 1) / sms;
   const int grid = (p->n + rpc - 1) / rpc;
-  const size_t vec = (size_t)NB * p->r * 4 + ((size_t)rpc / 32 + 2) * 4;
+  const size_t vec = pred2_vec_bytes(NB, p->r, rpc);
   int CR, NSL;
   used = ring_shape((size_t)p->r * sizeof(T), vec, ring2_budget(), rpc, CR, NSL);
   if (!used) return cudaSuccess;
@@ -1578,7 +1639,7 @@ cudaError_t run_down(const asf_ffn *f, int B, const int32_t *idx, const int32_t 
   const int S = down_splits(f);
   const size_t smem = (size_t)kWarps * NB * TW * 4;
   return launch(k_ffn_down<T, NB, 4>, dim3(ct, S), dim3(kThreads), smem, st, (const T *)f->WdT, a, idx, count,
-                f->d, ffn_rs(f), f->n, B, S, part, y, hdr, prefetch_enabled());
+                f->d, ffn_rs(f), f->n, B, S, part, y, hdr, prefetch_enabled(), l2_next_of(f));
 }
 
 // ------------------------------------------------------------- fused ffn --
@@ -1592,11 +1653,14 @@ int fused_nb(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 0; }
 // One CTA per SM (the ring's shared memory keeps a second one off each SM).
 int fused_grid() { return std::min(sm_count(), kMaxGrid); }
 
+// Most list positions one CTA of the grid takes.
+int fused_nl_max(const asf_ffn *f) { return (f->n + fused_grid() - 1) / fused_grid(); }
+
 // Ring slots that fit the shared-memory budget (0 if fewer than two).
 int fused_slots(const asf_ffn *f, int NB) {
   const int M = f->act == ASF_ACT_REGLU ? 3 : 2;
   for (int ns = 16; ns >= 2; --ns)
-    if (fused_layout(ns, f->d, M, esize(f->wdtype), NB).total <= fused_smem_budget()) return ns;
+    if (fused_layout(ns, f->d, M, esize(f->wdtype), NB, fused_nl_max(f)).total <= fused_smem_budget()) return ns;
   return 0;
 }
 
@@ -1615,7 +1679,7 @@ cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *i
   } else {
     const int M = REGLU ? 3 : 2;
     const int NS = fused_slots(f, NB);
-    const FusedLayout L = fused_layout(NS, f->d, M, (int)sizeof(T), NB);
+    const FusedLayout L = fused_layout(NS, f->d, M, (int)sizeof(T), NB, fused_nl_max(f));
     const int threads = (kFusedWarps + 1) * kWarp;
     auto kern = k_sparse_ffn<T, NB, MAXQ, REGLU>;
     const int G = fused_grid();
@@ -1624,7 +1688,7 @@ cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *i
                            idx ? std::max(0, f->hot_rows) : 0, ffn_rs(f), ffn_packed(f) ? 1 : 0, part, y, hdr);
     if (e != cudaSuccess) return e;
     return launch(k_reduce_partials, dim3((f->d + kWarp - 1) / kWarp, B), dim3(kReduceWarps * kWarp), 0, st,
-                  (const float *)part, G, B, f->d, y);
+                  (const float *)part, G, B, f->d, y, l2_next_of(f));
   }
 }
 
@@ -1737,7 +1801,7 @@ asf_status noalloc_scratch(void **out) {
 // ======================================================================== //
 extern "C" {
 
-int32_t asf_version(void) { return 102; }
+int32_t asf_version(void) { return 103; }
 
 const char *asf_status_string(asf_status s) {
   switch (s) {

@@ -81,13 +81,26 @@ class LayerStack:
         self.graph = None
 
 
-def build_layers(weights: List, device, hot_rows: Optional[Sequence[int]] = None) -> tuple:
+def build_layers(weights: List, device, hot_rows: Optional[Sequence[int]] = None,
+                 l2_next: bool = False) -> tuple:
     """Predictor and FFN descriptors for a list of ``synthetic.LayerWeights`` on ``device``.
 
     hot_rows[l] (optional) is the number of leading rows of layer l that the
-    offline profile found active for most tokens (the prefetch hint)."""
+    offline profile found active for most tokens (the prefetch hint).  With
+    l2_next, layer l's sparse FFN prefetches the predictor weights of layer
+    l+1 (of layer 0 after the last layer: the next token's first layer) into L2."""
     preds, ffns = [], []
     for l, w in enumerate(weights):
         preds.append(Predictor(w.W1, w.b1, w.W2, w.b2))
         ffns.append(FFN(w.act, w.Wg, w.Wu, w.WdT, w.bias, hot_rows=(hot_rows[l] if hot_rows else 0)))
+    if l2_next:
+        link_l2_next(preds, ffns)
     return preds, ffns
+
+
+def link_l2_next(preds: Sequence[Predictor], ffns: Sequence[FFN]) -> None:
+    """Point each layer's L2 hint at the next layer's predictor weights (cyclic)."""
+    L = len(ffns)
+    for l in range(L):
+        nxt = preds[(l + 1) % L]
+        ffns[l].set_l2_next(nxt.tensors[0], nxt.tensors[2])

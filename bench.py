@@ -47,6 +47,8 @@ def parse_args(argv=None):
                    help="FFN weight layout: neuron-major packed rows, or separate W_gate/W_up/W_down^T")
     p.add_argument("--no-hot-prefetch", action="store_true",
                    help="do not pass the hot-row prefetch hint to the sparse FFN")
+    p.add_argument("--l2-next", action="store_true",
+                   help="let each sparse FFN prefetch the next layer's predictor weights into L2")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=1024)
@@ -245,6 +247,7 @@ def workload_config(cfg, args):
             "weights": cfg.dtype, "accumulate": "f32",
             "l2": "inputs larger than L2: every step streams rows of all layers of a stack "
                   "whose weights exceed the 126 MB L2 many times over",
+            "l2_next": (args.mode == "predict" and args.l2_next),
             "parallelism": f"replicas x{args.gpus}"}
 
 
@@ -293,7 +296,7 @@ def run_ours(args, cfg):
     from activation_sparse_ffn_predict_b200 import build as _build
     _build.build()
     import activation_sparse_ffn_predict_b200 as A
-    from activation_sparse_ffn_predict_b200.stack import LayerStack, build_layers
+    from activation_sparse_ffn_predict_b200.stack import LayerStack, build_layers, link_l2_next
 
     from activation_sparse_ffn_predict_b200 import replicas as R
     ri = R.RankInfo.from_env()
@@ -316,6 +319,8 @@ def run_ours(args, cfg):
     L = cfg.layers
     T = args.tokens if args.tokens > 0 else cfg.tokens
     hot = cfg.hot_perm and not args.no_hot_perm
+    # each layer's sparse FFN pulls the next layer's predictor weights into L2
+    l2_next = args.mode == "predict" and args.l2_next
     weights, shares, hot_rows = [], [], []
     for l in range(L):
         w = S.layer_weights(cfg, l, device=device)
@@ -335,8 +340,10 @@ def run_ours(args, cfg):
             w.Wg = w.Wu = w.WdT = None      # the packed copy replaces the split matrices
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
+        if l2_next:
+            link_l2_next(preds, ffns)
     else:
-        preds, ffns = build_layers(weights, device, hot_rows if hot else None)
+        preds, ffns = build_layers(weights, device, hot_rows if hot else None, l2_next=l2_next)
     st = LayerStack(preds, ffns, B, cfg.tau, mode=args.mode, device=device)
     # token stream: each rank decodes its own tokens (replicas; no collectives)
     X = torch.empty(T, L, B, cfg.d, dtype=st.dtype, device=device)

@@ -102,6 +102,15 @@ typedef struct {
                          WdT = Wu + d) the layer is in the neuron-major packed layout
                          (gate|up|down of a neuron contiguous, see asf_gather_rows), and the
                          sparse FFN fetches each neuron with one bulk copy. */
+  const void *l2_next[2];      /* optional L2 prefetch hint: up to two device ranges that are
+                                  read soon after this call (for example the next layer's
+                                  predictor W1 and W2).  The call's last kernel pulls them into
+                                  L2 while it waits for the sparse FFN, whose row stream does
+                                  not keep HBM busy on its own.  Each non-NULL range must be
+                                  16-byte aligned and mapped for l2_next_bytes[i] bytes (the
+                                  tail below a multiple of 16 is skipped).  NULL / 0 = none.
+                                  Affects speed only, never results. */
+  int64_t l2_next_bytes[2];
 } asf_ffn;
 
 /* Bytes of device workspace needed by asf_predict / asf_sparse_ffn /
@@ -203,7 +212,8 @@ ASF_API asf_status asf_read_error(void *ws, int32_t *host_out, asf_stream_t stre
 /* Static description of a status code. */
 ASF_API const char *asf_status_string(asf_status s);
 
-/* ABI version: major * 100 + minor (1.02: asf_ffn.hot_rows, asf_ffn.row_stride, asf_gather_rows). */
+/* ABI version: major * 100 + minor (1.02: asf_ffn.hot_rows, asf_ffn.row_stride, asf_gather_rows;
+ * 1.03: asf_ffn.l2_next). */
 ASF_API int32_t asf_version(void);
 
 #ifdef __cplusplus

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.asf_version() == 102
+    assert lib.asf_version() == 103
     for code in range(8):
         assert lib.asf_status_string(code).decode() not in ("", "unknown status")
     assert lib.asf_status_string(99).decode() == "unknown status"
@@ -58,7 +58,7 @@ def test_struct_layout_matches_header():
     # int32 d, r, n; enum; then four pointers (8-byte aligned)
     assert ctypes.sizeof(L.asf_predictor) == 16 + 4 * 8
     assert L.asf_predictor.W1.offset == 16
-    assert ctypes.sizeof(L.asf_ffn) == 16 + 4 * 8 + 8   # + hot_rows, row_stride
+    assert ctypes.sizeof(L.asf_ffn) == 16 + 4 * 8 + 8 + 2 * 8 + 2 * 8   # + hot_rows, row_stride, l2_next[2], l2_next_bytes[2]
     assert L.asf_ffn.Wg.offset == 16
 
 
@@ -148,6 +148,13 @@ def test_sparse_ffn_rejects_bad_arguments(lib):
     assert _sparse(lib, f, y=FAKE + 8) == L.ASF_ERR_MISALIGNED
     need = lib.asf_workspace_bytes(None, ctypes.byref(f), 1)
     assert _sparse(lib, f, wsb=need - 1) == L.ASF_ERR_WORKSPACE
+    hinted = _ffn()
+    hinted.l2_next[1] = FAKE + 8
+    hinted.l2_next_bytes[1] = 4096
+    assert _sparse(lib, hinted) == L.ASF_ERR_MISALIGNED                # L2 hint not 16-byte aligned
+    hinted.l2_next[1] = FAKE
+    hinted.l2_next_bytes[1] = -16
+    assert _sparse(lib, hinted) == L.ASF_ERR_INVALID_ARG
     assert lib.asf_dense_ffn(ctypes.byref(f), FAKE, 1, FAKE, FAKE, need - 1, None) == L.ASF_ERR_WORKSPACE
     assert lib.asf_dense_ffn(ctypes.byref(f), FAKE, 0, FAKE, FAKE, need, None) == L.ASF_ERR_INVALID_ARG
 

@@ -255,6 +255,38 @@ def test_hot_row_hint_changes_nothing_but_speed(layer):
     assert layer.error() == 0
 
 
+def test_l2_next_hint_changes_nothing_but_speed(layer):
+    # The hint makes the call's last kernel prefetch other ranges into L2:
+    # results of both FFN paths (fused at B <= 4, two-kernel above) and of a
+    # dense call are bit-identical with it, and no device error is raised.
+    cfg = layer.cfg
+    w = layer.w
+    hinted = A.FFN(w.act, w.Wg, w.Wu, w.WdT, w.bias)
+    hinted.set_l2_next(w.W1, w.W2)
+    odd = torch.empty(4 * 1024 + 48, dtype=torch.uint8, device="cuda")    # not a multiple of 16 bytes long
+    for B in (1, 3, 16):
+        rows = slice(0, B)
+        idx = layer.oracle_idx(rows)
+        x = layer.Xd[rows].contiguous()
+        idt = torch.zeros(cfg.n, dtype=torch.int32, device="cuda")
+        if idx.size:
+            idt[:idx.size] = torch.from_numpy(idx).cuda()
+        cnt = torch.tensor([idx.size], dtype=torch.int32, device="cuda")
+        y0 = torch.zeros(B, cfg.d, dtype=torch.float32, device="cuda")
+        y1 = torch.zeros(B, cfg.d, dtype=torch.float32, device="cuda")
+        A.asf_sparse_ffn(layer.ffn, x, idt, cnt, y0, layer.ws)
+        A.asf_sparse_ffn(hinted, x, idt, cnt, y1, layer.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y0, y1)
+        hinted.set_l2_next(odd[:4 * 1024 + 40])
+        A.asf_dense_ffn(layer.ffn, x, y0, layer.ws)
+        A.asf_dense_ffn(hinted, x, y1, layer.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y0, y1)
+        hinted.set_l2_next(w.W1, w.W2)
+    assert layer.error() == 0
+
+
 def test_packed_layout_is_bitwise_equal_to_split_layout(layer):
     # Neuron-major packed rows (one bulk copy per neuron) change the memory
     # layout only: every FFN path must give bit-identical results.

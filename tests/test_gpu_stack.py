@@ -15,9 +15,10 @@ from activation_sparse_ffn_predict_b200.stack import LayerStack, build_layers
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B", [1, 4])
-@pytest.mark.parametrize("mode", ["predict", "dense"])
-def test_graph_stack_matches_oracle(B, mode):
+@pytest.mark.parametrize("B,mode,l2_next", [(1, "predict", False), (4, "predict", False),
+                                            (1, "dense", False), (4, "dense", False),
+                                            (1, "predict", True), (12, "predict", True)])
+def test_graph_stack_matches_oracle(B, mode, l2_next):
     ensure_built()
     cfg = S.get("llama2_7b_reglu").with_(d=1024, n=2752, r=128, layers=3)
     tokens = 3 * B
@@ -31,7 +32,7 @@ def test_graph_stack_matches_oracle(B, mode):
         hosts.append(h)
         devs.append(w.to("cuda"))
         xs.append(X)
-    preds, ffns = build_layers(devs, "cuda")
+    preds, ffns = build_layers(devs, "cuda", l2_next=l2_next)
     st = LayerStack(preds, ffns, B, cfg.tau, mode=mode)
     st.capture()
     for step in range(3):

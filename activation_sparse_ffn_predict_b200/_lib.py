@@ -44,6 +44,8 @@ PROTOTYPES = {
                             c_void_p, c_size_t, c_void_p]),
     "asf_sparse_ffn": (c_int, [POINTER(asf_ffn), c_void_p, c_int32, c_void_p, c_void_p, c_void_p,
                                c_void_p, c_size_t, c_void_p]),
+    "asf_predict_sparse_ffn": (c_int, [POINTER(asf_predictor), POINTER(asf_ffn), c_void_p, c_int32, c_float,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "asf_dense_ffn": (c_int, [POINTER(asf_ffn), c_void_p, c_int32, c_void_p, c_void_p, c_size_t,
                               c_void_p]),
     "asf_activation_counts": (c_int, [POINTER(asf_ffn), c_void_p, c_int32, c_void_p, c_void_p,

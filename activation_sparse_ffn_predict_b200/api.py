@@ -172,6 +172,21 @@ def asf_sparse_ffn(ffn: FFN, x: torch.Tensor, idx: torch.Tensor, count: torch.Te
     check(st, "asf_sparse_ffn")
 
 
+def asf_predict_sparse_ffn(pred: Predictor, ffn: FFN, x: torch.Tensor, tau: float, idx: torch.Tensor,
+                           count: torch.Tensor, y: torch.Tensor, ws: Workspace, stream=None) -> None:
+    """One layer: asf_predict then asf_sparse_ffn over the predicted list, in
+    one call (same idx, count and y); ws must be sized with both descriptors."""
+    if x.dtype != ffn.dtype or x.dim() != 2 or x.shape[1] != ffn.d:
+        raise ValueError("x must be [B, d] in the FFN's dtype")
+    if y.shape != (x.shape[0], ffn.d):
+        raise ValueError("y must be [B, d]")
+    st = L.load().asf_predict_sparse_ffn(ctypes.byref(pred.desc), ctypes.byref(ffn.desc), _dev(x, "x"),
+                                         int(x.shape[0]), float(tau), _dev(idx, "idx", torch.int32),
+                                         _dev(count, "count", torch.int32), _dev(y, "y", torch.float32),
+                                         ws.ptr, ws.nbytes, _stream(stream))
+    check(st, "asf_predict_sparse_ffn")
+
+
 def asf_sparse_ffn_noalloc(ffn: FFN, x: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
                            y: torch.Tensor, fault: Optional[torch.Tensor] = None, stream=None) -> None:
     """asf_sparse_ffn without a workspace: for callers that cannot allocate

@@ -202,22 +202,18 @@ template <typename T, int NB, int U>
 __global__ void __launch_bounds__(kThreads)
     k_pred_l1(const T *__restrict__ W1, const float *__restrict__ b1, const T *__restrict__ x, int d,
               int r, int B, int rpc, float *__restrict__ h, uint32_t *__restrict__ mask_words,
-              int n_words, const T *__restrict__ W2, int n, int prefetch) {
+              int n_words) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   T *xs = reinterpret_cast<T *>(smem_raw);
   constexpr int V = Vec<T>::N;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row0 = blockIdx.x * rpc;
   const int row1 = min(r, row0 + rpc);
-  if (prefetch) {
-    // this CTA's W1 rows, and its share of W2 for the second predictor layer:
-    // both stream into L2 while the previous kernel is still running
-    if (row0 < row1) prefetch_range(W1 + (size_t)row0 * d, (size_t)(row1 - row0) * d * sizeof(T));
-    const int w0 = (int)(((long long)n * blockIdx.x) / gridDim.x);
-    const int w1 = (int)(((long long)n * (blockIdx.x + 1)) / gridDim.x);
-    if (w0 < w1) prefetch_range(W2 + (size_t)w0 * r, (size_t)(w1 - w0) * r * sizeof(T));
-  }
-  // The next kernel reads only weights before it waits on this one.
+  // No L2 prefetch here: this grid becomes resident while the previous
+  // layer's sparse FFN starts its row stream, and weight traffic issued now
+  // would delay those rows (the asf_ffn.l2_next hint prefetches the weights
+  // once the rows are queued).  The next kernel reads only weights before it
+  // waits on this one.
   pdl_trigger();
   pdl_wait();
   for (int w = blockIdx.x * kThreads + threadIdx.x; w < n_words; w += gridDim.x * kThreads)
@@ -417,7 +413,7 @@ __device__ __forceinline__ void ring_issue(const T *W, int K, int row0, int row1
   const int rb = min(row1, ra + CR);
   const uint32_t bytes = (uint32_t)((size_t)(rb - ra) * K * sizeof(T));
   mbar_arrive_expect_tx(&full[s], bytes);
-  bulk_g2s(ring + (size_t)s * CR * K, W + (size_t)ra * K, bytes, &full[s]);
+  bulk_g2s_stream(ring + (size_t)s * CR * K, W + (size_t)ra * K, bytes, &full[s], l2_evict_first());
 }
 
 // Producer loop for chunks [first, nch): waits for slot release, then issues.
@@ -430,92 +426,6 @@ __device__ __forceinline__ bool ring_produce(const T *W, int K, int row0, int ro
     ring_issue(W, K, row0, row1, CR, NSL, i, ring, full);
   }
   return true;
-}
-
-// Layer 1 of the predictor, B <= NB tokens: h = max(W1 x + b1, 0).  CTA c's
-// rows [c*rpc, (c+1)*rpc) are contiguous in memory; the producer warp copies
-// them in chunks of CR rows into an NSL-slot ring, the first chunks before the
-// kernel waits on its predecessor (weights do not depend on it).  It also
-// L2-prefetches this CTA's share of W2 for the second layer.
-template <typename T, int NB>
-__global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
-    k_pred1_ring(const T *__restrict__ W1, const float *__restrict__ b1, const T *__restrict__ x, int d, int r,
-                 int B, int rpc, int CR, int NSL, float *__restrict__ h, uint32_t *__restrict__ mask_words,
-                 int n_words, const T *__restrict__ W2, int n, int32_t *__restrict__ err, int prefetch) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int V = Vec<T>::N;
-  const RingLayout L = ring_layout(NSL, CR, d, (int)sizeof(T), (size_t)NB * d * sizeof(T));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
-  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + L.empty);
-  T *xs = reinterpret_cast<T *>(smem + L.vec);
-  T *ring = reinterpret_cast<T *>(smem + L.ring);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = blockIdx.x * rpc, row1 = min(r, row0 + rpc);
-  const int nch = row0 < row1 ? (row1 - row0 + CR - 1) / CR : 0;
-  if (threadIdx.x == 0) {
-    for (int q = 0; q < NSL; ++q) {
-      mbar_init(&full[q], 1);
-      mbar_init(&empty[q], kRingWarps);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (warp == kRingWarps && lane == 0) {
-    for (int i = 0; i < min(nch, NSL); ++i) ring_issue(W1, d, row0, row1, CR, NSL, i, ring, full);
-  }
-  if (prefetch && warp == kRingWarps) {
-    const int w0 = (int)(((long long)n * blockIdx.x) / gridDim.x);
-    const int w1 = (int)(((long long)n * (blockIdx.x + 1)) / gridDim.x);
-    if (w0 < w1) {
-      const size_t bytes = (size_t)(w1 - w0) * r * sizeof(T);
-      const unsigned char *base = reinterpret_cast<const unsigned char *>(W2 + (size_t)w0 * r);
-      for (size_t o = (size_t)lane * 16384; o < bytes; o += 32 * 16384)
-        prefetch_l2(base + o, (uint32_t)min((size_t)16384, bytes - o));
-    }
-  }
-  // the next kernel reads only weights before it waits on this one
-  pdl_trigger();
-  pdl_wait();
-  for (int w = blockIdx.x * blockDim.x + threadIdx.x; w < n_words; w += gridDim.x * blockDim.x) mask_words[w] = 0u;
-  if (warp == kRingWarps) {
-    if (lane == 0 && !ring_produce(W1, d, row0, row1, CR, NSL, NSL, nch, ring, full, empty))
-      flag_error(err, kErrTimeout);
-  } else {
-    const int nvec = d / V;
-    stage16<8>(reinterpret_cast<uint4 *>(xs), reinterpret_cast<const uint4 *>(x), B * nvec, kRingWarps * kWarp);
-    for (int i = B * nvec + threadIdx.x; i < NB * nvec; i += kRingWarps * kWarp)
-      reinterpret_cast<uint4 *>(xs)[i] = make_uint4(0u, 0u, 0u, 0u);
-    named_sync(1, kRingWarps * kWarp);
-    bool ok = true;
-    for (int i = 0; i < nch; ++i) {
-      const int sl = i % NSL;
-      if (ok && !mbar_wait(&full[sl], (uint32_t)(i / NSL) & 1u, kWaitNs)) {
-        if (lane == 0) flag_error(err, kErrTimeout);
-        ok = false;
-      }
-      const int ra = row0 + i * CR, rb = min(row1, ra + CR);
-      for (int row = ra + warp; row < rb && ok; row += kRingWarps) {
-        const T *wr = ring + ((size_t)sl * CR + (row - ra)) * d;
-        float acc[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-        for (int c = lane; c < nvec; c += kWarp) {
-          const uint4 wv = *reinterpret_cast<const uint4 *>(wr + (size_t)c * V);
-#pragma unroll
-          for (int b = 0; b < NB; ++b)
-            acc[b] = Vec<T>::dot(wv, *reinterpret_cast<const uint4 *>(xs + (size_t)b * d + (size_t)c * V), acc[b]);
-        }
-        const float bias = __ldg(b1 + row);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const float sum = warp_sum(acc[b]);
-          if (lane == b && b < B) h[(size_t)b * r + row] = fmaxf(sum + bias, 0.f);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[sl]);
-    }
-  }
 }
 
 // Shared bytes of k_pred2_ring besides the ring: staged h [NB][r], the CTA's
@@ -913,11 +823,13 @@ __global__ void __launch_bounds__(kThreads)
 // Shared-memory layout of k_sparse_ffn for NS ring slots of M rows of d elements.
 struct FusedLayout {
   int NS, grp;
-  size_t full, empty, kslot, bias, pd, x, stage, red, total;
+  size_t full, empty, kslot, list, bias, words, pd, x, stage, red, total;
 };
 
-// nl_max: most list positions one CTA takes (ceil(n / grid)).
-__host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int esz, int NB, int nl_max) {
+// nl_max: most list positions one CTA takes (ceil(n / grid)); mask_words:
+// words of the union mask the kernel ranks itself (0 when it gets a list).
+__host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int esz, int NB, int nl_max,
+                                                    int mask_words) {
   FusedLayout L;
   L.NS = NS;
   L.grp = NS / 2 > 0 ? NS / 2 : 1;
@@ -925,7 +837,10 @@ __host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int es
   L.full = o;  o += (size_t)NS * 8;
   L.empty = o; o += (size_t)NS * 8;
   L.kslot = o; o += (size_t)NS * 4;
+  L.list = o;  o += (size_t)nl_max * 4;
   L.bias = o;  o += (size_t)nl_max * 4;
+  o = align_up(o, 16);
+  L.words = o; o += (size_t)(mask_words + 3) / 4 * 16 * 2;    // the words, then their prefix counts
   o = align_up(o, 16);
   L.pd = o;    o += (size_t)kFusedWarps * L.grp * 2 * NB * 4;
   o = align_up(o, 128);
@@ -937,9 +852,81 @@ __host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int es
   return L;
 }
 
+// The ascending list of the set bits of a union mask (n bits in n_words
+// words), as one CTA of G needs it: slist[i] = the bit at list position
+// c + i*G.  One warp.  The words are staged in shared memory (sw, 16-byte
+// aligned, n_words rounded up to 4); each lane takes a contiguous block of
+// words and, after a warp scan of the blocks' popcounts, writes every word's
+// inclusive prefix count (spre).  Then each lane takes list positions and
+// finds its word by binary search over spre and the bit within it.  Returns
+// the number of set bits.
+__device__ __forceinline__ int list_from_mask(const uint32_t *__restrict__ mask, int n_words, int n, int c, int G,
+                                              int *slist, uint32_t *sw, int *spre) {
+  constexpr int MAXU = 4;
+  const int lane = threadIdx.x & 31;
+  const int nq = (n_words + 3) / 4;               // 16-byte groups of words
+  const uint32_t tail = (n & 31) ? ((1u << (n & 31)) - 1u) : 0xffffffffu;
+  for (int q0 = 0; q0 < nq; q0 += MAXU * kWarp) {
+    uint4 v[MAXU];
+#pragma unroll
+    for (int u = 0; u < MAXU; ++u) {
+      const int q = q0 + u * kWarp + lane;
+      v[u] = q < nq ? __ldcg(reinterpret_cast<const uint4 *>(mask) + q) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < MAXU; ++u) {
+      const int q = q0 + u * kWarp + lane;
+      if (q < nq) {
+        uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int w = 4 * q + e;
+          w4[e] = w < n_words ? (w == n_words - 1 ? (w4[e] & tail) : w4[e]) : 0u;
+        }
+        reinterpret_cast<uint4 *>(sw)[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    }
+  }
+  __syncwarp();
+  const int per = (n_words + kWarp - 1) / kWarp;
+  const int wb = min(n_words, lane * per), we = min(n_words, wb + per);
+  int tot = 0;
+  for (int w = wb; w < we; ++w) tot += __popc(sw[w]);
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < kWarp; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int cnt = __shfl_sync(0xffffffffu, incl, kWarp - 1);
+  int run = incl - tot;
+  for (int w = wb; w < we; ++w) {
+    run += __popc(sw[w]);
+    spre[w] = run;
+  }
+  __syncwarp();
+  const int nl = cnt > c ? (cnt - 1 - c) / G + 1 : 0;
+  for (int i = lane; i < nl; i += kWarp) {
+    const int p = c + G * i;
+    int lo = 0, hi = n_words - 1;          // first word whose inclusive count exceeds p
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (spre[mid] > p) hi = mid; else lo = mid + 1;
+    }
+    uint32_t m = sw[lo];
+    for (int q = p - (lo ? spre[lo - 1] : 0); q > 0; --q) m &= m - 1u;   // drop the lower set bits
+    slist[i] = lo * 32 + __ffs(m) - 1;
+  }
+  return cnt;
+}
+
 // One kernel for the whole neuron-sparse FFN of B <= NB tokens.
 //
-// CTA c of a grid of G takes list positions [c*cnt/G, (c+1)*cnt/G).  Warp
+// CTA c of a grid of G takes list positions c, c + G, c + 2G, ...: its first
+// index loads need not wait for the count.  The list comes from idx/count, or
+// (idx == NULL) is every neuron, or (mask != NULL) is built here from the
+// predictor's union mask, whose set bits this kernel ranks itself and writes
+// out as idx_out/count_out (no separate compaction kernel).  Warp
 // kFusedWarps is the producer: one lane streams, for each of its neurons k,
 // the rows Wg[k], Wu[k], WdT[k] into a ring of NS shared-memory slots with
 // cp.async.bulk, completing on the slot's "full" mbarrier.  The 8 consumer
@@ -951,23 +938,29 @@ __host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int es
 // a * WdT[k] into its registers; then it releases the slot ("empty").
 // At the end every CTA stores its y partial; k_reduce_partials, the next
 // kernel, sums them in a fixed order (deterministic, no float atomics).
+// Once the producer has queued its last copy it issues this CTA's share of the
+// asf_ffn.l2_next L2 prefetch.
 template <typename T, int NB, int MAXQ, bool REGLU>
 __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     k_sparse_ffn(const T *__restrict__ Wg, const T *__restrict__ Wu, const T *__restrict__ WdT,
                  const float *__restrict__ bias, const T *__restrict__ x, int d, int n, int B,
-                 const int32_t *__restrict__ idx, const int32_t *__restrict__ count, int NS, int hot_rows,
+                 const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
+                 const uint32_t *__restrict__ mask, int n_words, int32_t *__restrict__ idx_out,
+                 int32_t *__restrict__ count_out, int NS, int hot_rows,
                  long long rs, int packed, float *__restrict__ part, float *__restrict__ y,
-                 Header *__restrict__ hdr) {
+                 Header *__restrict__ hdr, L2Next nx) {
   constexpr int V = Vec<T>::N;
   constexpr int M = REGLU ? 3 : 2;
   constexpr int NW = kFusedWarps;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_fail;
-  const FusedLayout L = fused_layout(NS, d, M, (int)sizeof(T), NB, (n + (int)gridDim.x - 1) / (int)gridDim.x);
+  __shared__ int s_fail, s_nl;
+  const FusedLayout L = fused_layout(NS, d, M, (int)sizeof(T), NB, (n + (int)gridDim.x - 1) / (int)gridDim.x,
+                                     mask ? n_words : 0);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
   uint64_t *empty = reinterpret_cast<uint64_t *>(smem + L.empty);
   int *kslot = reinterpret_cast<int *>(smem + L.kslot);
-  float *sbias = reinterpret_cast<float *>(smem + L.bias);    // bias of list position js + i
+  int *slist = reinterpret_cast<int *>(smem + L.list);        // neuron at list position c + i*G
+  float *sbias = reinterpret_cast<float *>(smem + L.bias);    // its bias
   float *pd = reinterpret_cast<float *>(smem + L.pd);
   T *xs = reinterpret_cast<T *>(smem + L.x);
   T *stage = reinterpret_cast<T *>(smem + L.stage);
@@ -1006,19 +999,7 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
   pdl_trigger();
   pdl_wait();
 
-  int cnt = n;
-  if (idx) {
-    const int c = ld_cg_i32(count);
-    if (c < 0 || c > n) {
-      if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(err, kErrIndex);
-    }
-    cnt = max(0, min(c, n));
-  }
-  const int G = gridDim.x;
-  const int js = (int)(((long long)cnt * blockIdx.x) / G);
-  const int je = (int)(((long long)cnt * (blockIdx.x + 1)) / G);
-  const int nl = je - js;
-
+  const int G = gridDim.x, cta = blockIdx.x;
   float acc[MAXQ][V][NB];
 #pragma unroll
   for (int q = 0; q < MAXQ; ++q)
@@ -1028,24 +1009,59 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
       for (int b = 0; b < NB; ++b) acc[q][e][b] = 0.f;
 
   if (warp == NW) {
+    // -------------------------------------------------- this CTA's list --
+    int cnt;
+    if (mask) {
+      uint32_t *sw = reinterpret_cast<uint32_t *>(smem + L.words);
+      cnt = list_from_mask(mask, n_words, n, cta, G, slist, sw, reinterpret_cast<int *>(sw) + (n_words + 3) / 4 * 4);
+    } else if (idx) {
+      // the count and the first 32 positions are fetched together
+      const int p0 = cta + G * lane;
+      const int c_raw = ld_cg_i32(count);
+      const int k0 = p0 < n ? ld_cg_i32(idx + p0) : -1;
+      if ((c_raw < 0 || c_raw > n) && cta == 0 && lane == 0) flag_error(err, kErrIndex);
+      cnt = max(0, min(c_raw, n));
+      const int nl0 = cnt > cta ? (cnt - 1 - cta) / G + 1 : 0;
+      if (lane < nl0) slist[lane] = k0;
+      for (int i = kWarp + lane; i < nl0; i += kWarp) slist[i] = ld_cg_i32(idx + cta + (size_t)G * i);
+    } else {
+      cnt = n;
+      const int nl0 = n > cta ? (n - 1 - cta) / G + 1 : 0;
+      for (int i = lane; i < nl0; i += kWarp) slist[i] = cta + G * i;
+    }
+    if (lane == 0) s_nl = cnt > cta ? (cnt - 1 - cta) / G + 1 : 0;
+    // hand the list to the consumers without waiting for them
+    __syncwarp();
+    named_arrive(2, (NW + 1) * kWarp);
+    if (mask && lane > 0) {
+      // this CTA's positions of the list, written out by the lanes that do
+      // not issue copies (all CTAs together write idx_out[0..count))
+      const int nlp = s_nl;
+      for (int i = lane - 1; i < nlp; i += kWarp - 1) idx_out[cta + (size_t)G * i] = slist[i];
+      if (cta == 0 && lane == 1) *count_out = cnt;
+    }
+  } else {
+    // consumers: x into shared memory while the list is being fetched
+    stage16<8>(reinterpret_cast<uint4 *>(xs), reinterpret_cast<const uint4 *>(x), B * nvec, NW * kWarp);
+    for (int i = B * nvec + threadIdx.x; i < NB * nvec; i += NW * kWarp)
+      reinterpret_cast<uint4 *>(xs)[i] = make_uint4(0u, 0u, 0u, 0u);
+    named_sync(2, (NW + 1) * kWarp);
+  }
+  const int nl = s_nl;
+
+  if (warp == NW) {
     // ------------------------------------------------------------ producer --
-    // The whole warp walks the list; indices are fetched 32 at a time with one
-    // coalesced load and broadcast by shuffle; lane 0 issues the copies.
+    // lane 0 issues one neuron's copies per ring slot
     const uint32_t row_bytes = (uint32_t)((size_t)d * sizeof(T));
-    int kreg = 0;
-    bool stop = false;
-    for (int i = 0; i < nl && !stop; ++i) {
-      if ((i & 31) == 0) {
-        const int j = js + i + lane;
-        kreg = (j < je) ? (idx ? ld_cg_i32(idx + j) : j) : -1;
-      }
-      const int k = __shfl_sync(0xffffffffu, kreg, i & 31);
-      if (lane == 0) {
+    const uint64_t pol = l2_evict_first();
+    for (int i = 0; i < nl && lane == 0; ++i) {
+      const int k = slist[i];
+      {
         const int s = i % NS;
         if (i >= NS && !mbar_wait(&empty[s], (uint32_t)((i / NS) - 1) & 1u, kWaitNs)) {
           flag_error(err, kErrTimeout);
           s_fail = 1;
-          stop = true;
+          break;
         } else if ((unsigned)k >= (unsigned)n) {
           flag_error(err, kErrIndex);
           kslot[s] = -1;
@@ -1055,27 +1071,28 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
           mbar_arrive_expect_tx(&full[s], (uint32_t)M * row_bytes);
           T *dst = stage + (size_t)s * M * d;
           if (packed) {          // the neuron's rows are one contiguous block
-            bulk_g2s(dst, (REGLU ? Wg : Wu) + (size_t)k * rs, (uint32_t)M * row_bytes, &full[s]);
+            bulk_g2s_stream(dst, (REGLU ? Wg : Wu) + (size_t)k * rs, (uint32_t)M * row_bytes, &full[s], pol);
           } else if constexpr (REGLU) {
-            bulk_g2s(dst, Wg + (size_t)k * rs, row_bytes, &full[s]);
-            bulk_g2s(dst + d, Wu + (size_t)k * rs, row_bytes, &full[s]);
-            bulk_g2s(dst + 2 * (size_t)d, WdT + (size_t)k * rs, row_bytes, &full[s]);
+            bulk_g2s_stream(dst, Wg + (size_t)k * rs, row_bytes, &full[s], pol);
+            bulk_g2s_stream(dst + d, Wu + (size_t)k * rs, row_bytes, &full[s], pol);
+            bulk_g2s_stream(dst + 2 * (size_t)d, WdT + (size_t)k * rs, row_bytes, &full[s], pol);
           } else {
-            bulk_g2s(dst, Wu + (size_t)k * rs, row_bytes, &full[s]);
-            bulk_g2s(dst + d, WdT + (size_t)k * rs, row_bytes, &full[s]);
+            bulk_g2s_stream(dst, Wu + (size_t)k * rs, row_bytes, &full[s], pol);
+            bulk_g2s_stream(dst + d, WdT + (size_t)k * rs, row_bytes, &full[s], pol);
           }
         }
       }
-      stop = __shfl_sync(0xffffffffu, stop, 0);
     }
+    __syncwarp();
+    // Every row copy of this CTA is queued: only now pull the hinted ranges
+    // into L2, so that they take bandwidth the row stream leaves idle instead
+    // of delaying its first rows.
+    prefetch_next(nx, blockIdx.x, gridDim.x);
   } else {
     // ----------------------------------------------------------- consumers --
-    stage16<8>(reinterpret_cast<uint4 *>(xs), reinterpret_cast<const uint4 *>(x), B * nvec, NW * kWarp);
-    for (int i = B * nvec + threadIdx.x; i < NB * nvec; i += NW * kWarp)
-      reinterpret_cast<uint4 *>(xs)[i] = make_uint4(0u, 0u, 0u, 0u);
     // the biases of this CTA's neurons, while the first rows are in flight
     for (int i = threadIdx.x; i < nl; i += NW * kWarp) {
-      const int k = idx ? ld_cg_i32(idx + js + i) : js + i;
+      const int k = slist[i];
       sbias[i] = (unsigned)k < (unsigned)n ? __ldg(bias + k) : 0.f;
     }
     named_sync(1, NW * kWarp);
@@ -1203,12 +1220,9 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
 constexpr int kReduceWarps = 8;
 constexpr int kReduceMaxPerWarp = 32;   // G <= 256
 __global__ void __launch_bounds__(kReduceWarps * kWarp)
-    k_reduce_partials(const float *__restrict__ part, int G, int B, int d, float *__restrict__ y, L2Next nx) {
+    k_reduce_partials(const float *__restrict__ part, int G, int B, int d, float *__restrict__ y) {
   __shared__ float red[kReduceWarps][kWarp];
   pdl_trigger();
-  // This grid starts while the sparse FFN still streams its rows; the hinted
-  // ranges fill L2 in that time.
-  if (threadIdx.x < kWarp) prefetch_next(nx, blockIdx.y * gridDim.x + blockIdx.x, gridDim.x * gridDim.y);
   pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int col = blockIdx.x * kWarp + lane;
@@ -1474,8 +1488,7 @@ cudaError_t run_pred_l1(const asf_predictor *p, const void *x, int B, float *h, 
   const int grid = (p->r + rpc - 1) / rpc;
   const size_t smem = (size_t)NB * p->d * sizeof(T);
   return launch(k_pred_l1<T, NB, (NB <= 2 ? 16 : 8)>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W1, p->b1,
-                (const T *)x, p->d, p->r, B, rpc, h, mask, n_words_of(p->n), (const T *)p->W2, p->n,
-                prefetch_enabled());
+                (const T *)x, p->d, p->r, B, rpc, h, mask, n_words_of(p->n));
 }
 
 template <typename T, int NB>
@@ -1490,14 +1503,12 @@ cudaError_t run_pred_l2(const asf_predictor *p, int B, float thr, const float *h
 }
 
 constexpr size_t kRingChunk = 32 * 1024;    // bytes per bulk copy of a ring slot
-constexpr size_t kRing1Smem = 80 * 1024;     // layer-1 ring + x
+// Shared memory of the layer-2 ring: with the register-streaming layer-1
+// kernel (one token group of x) it fits beside the previous layer's sparse
+// FFN tail, and it holds most of a CTA's W2 slice.
 size_t ring2_budget() {
   static size_t kb = (size_t)env_flag("ASFFN_RING2_KB", 136);
   return std::min<size_t>(std::max<size_t>(kb, 40), 200) * 1024;
-}
-bool ring1_enabled() {
-  static int on = env_flag("ASFFN_RING1", 0);
-  return on != 0;
 }
 
 // rows per chunk and slots for a ring over rows of row_bytes within budget
@@ -1508,21 +1519,6 @@ bool ring_shape(size_t row_bytes, size_t vec_bytes, size_t budget, int rpc, int 
   for (NSL = std::min(8, std::max(chunks, 2)); NSL >= 2; --NSL)
     if (ring_layout(NSL, CR, 1, (int)row_bytes, vec_bytes).total <= budget) return true;
   return false;
-}
-
-template <typename T, int NB>
-cudaError_t run_pred1_ring(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, int32_t *err,
-                           cudaStream_t st, bool &used) {
-  const int sms = sm_count();
-  const int rpc = (p->r + sms - 1) / sms;
-  const int grid = (p->r + rpc - 1) / rpc;
-  int CR, NSL;
-  used = ring_shape((size_t)p->d * sizeof(T), (size_t)NB * p->d * sizeof(T), kRing1Smem, rpc, CR, NSL);
-  if (!used) return cudaSuccess;
-  const size_t smem = ring_layout(NSL, CR, p->d, (int)sizeof(T), (size_t)NB * p->d * sizeof(T)).total;
-  return launch(k_pred1_ring<T, NB>, dim3(grid), dim3((kRingWarps + 1) * kWarp), smem, st, (const T *)p->W1,
-                p->b1, (const T *)x, p->d, p->r, B, rpc, CR, NSL, h, mask, n_words_of(p->n), (const T *)p->W2,
-                p->n, err, prefetch_enabled());
 }
 
 template <typename T, int NB>
@@ -1549,17 +1545,6 @@ bool ring_enabled() {
 
 // largest token group in {1, 2, 4, 8} covering B (B <= 8)
 inline int nb_cover(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 8; }
-
-template <typename T>
-cudaError_t pred1_ring_any(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, int32_t *err,
-                           cudaStream_t st, bool &used) {
-  switch (nb_cover(B)) {
-    case 1: return run_pred1_ring<T, 1>(p, x, B, h, mask, err, st, used);
-    case 2: return run_pred1_ring<T, 2>(p, x, B, h, mask, err, st, used);
-    case 4: return run_pred1_ring<T, 4>(p, x, B, h, mask, err, st, used);
-    default: return run_pred1_ring<T, 8>(p, x, B, h, mask, err, st, used);
-  }
-}
 
 template <typename T>
 cudaError_t pred2_ring_any(const asf_predictor *p, int B, float thr, const float *h, uint32_t *mask, int32_t *idx,
@@ -1593,9 +1578,27 @@ cudaError_t pred2_reg_any(const asf_predictor *p, int B, float thr, const float 
   }
 }
 
-// Layer 1 then layer 2 + compaction.  Batches of up to 8 tokens use the
-// bulk-copy ring kernels when their slices fit; larger batches use the
-// register-streaming kernels, which loop over token groups.
+// Layer 1 (register-streaming kernel, token groups of up to 8), then layer 2:
+// batches of up to 8 tokens use the bulk-copy ring kernel followed by the
+// compaction kernel when the slice fits; larger batches use the
+// register-streaming layer-2 kernel, which compacts in its last CTA.
+template <typename T>
+cudaError_t predict_layers(const asf_predictor *p, const void *x, int B, float thr, int32_t *idx, int32_t *count,
+                           Header *hdr, uint32_t *mask, float *h, cudaStream_t st, bool &mask_only) {
+  const bool ring = B <= 8 && ring_enabled() && n_words_of(p->n) <= kCompactThreads * kCompactWords;
+  mask_only = false;
+  cudaError_t e = pred1_reg_any<T>(p, x, B, h, mask, st);
+  if (e != cudaSuccess) return e;
+  if (ring) e = pred2_ring_any<T>(p, B, thr, h, mask, idx, count, hdr, st, mask_only);
+  if (e != cudaSuccess || mask_only) return e;   // mask_only: the ring kernel left the union mask
+  return pred2_reg_any<T>(p, B, thr, h, mask, idx, count, hdr, st);
+}
+
+cudaError_t launch_compact(const asf_predictor *p, const uint32_t *mask, int32_t *idx, int32_t *count,
+                           cudaStream_t st) {
+  return launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, mask, n_words_of(p->n), idx, count);
+}
+
 template <typename T>
 asf_status predict_t(const asf_predictor *p, const void *x, int B, float thr, int32_t *idx, int32_t *count,
                      void *ws, cudaStream_t st) {
@@ -1603,19 +1606,10 @@ asf_status predict_t(const asf_predictor *p, const void *x, int B, float thr, in
   Header *hdr = reinterpret_cast<Header *>(base);
   uint32_t *mask = reinterpret_cast<uint32_t *>(base + kHeaderBytes);
   float *h = reinterpret_cast<float *>(base + kHeaderBytes + mask_region(p));
-  const bool ring = B <= 8 && ring_enabled() && n_words_of(p->n) <= kCompactThreads * kCompactWords;
-  bool used = false;
-  cudaError_t e = cudaSuccess;
-  if (ring && ring1_enabled()) e = pred1_ring_any<T>(p, x, B, h, mask, &hdr->err, st, used);
-  if (e == cudaSuccess && !used) e = pred1_reg_any<T>(p, x, B, h, mask, st);
-  if (e != cudaSuccess) return ASF_ERR_CUDA;
-  used = false;
-  if (ring) e = pred2_ring_any<T>(p, B, thr, h, mask, idx, count, hdr, st, used);
-  if (e != cudaSuccess) return ASF_ERR_CUDA;
-  if (used)   // the ring kernel leaves the union mask; compact it
-    return cuda_status(launch(k_compact, dim3(1), dim3(kCompactThreads), 0, st, (const uint32_t *)mask,
-                              n_words_of(p->n), idx, count));
-  return cuda_status(pred2_reg_any<T>(p, B, thr, h, mask, idx, count, hdr, st));
+  bool mask_only = false;
+  cudaError_t e = predict_layers<T>(p, x, B, thr, idx, count, hdr, mask, h, st, mask_only);
+  if (e == cudaSuccess && mask_only) e = launch_compact(p, mask, idx, count, st);
+  return cuda_status(e);
 }
 
 // ------------------------------------------------------------------- ffn --
@@ -1657,10 +1651,11 @@ int fused_grid() { return std::min(sm_count(), kMaxGrid); }
 int fused_nl_max(const asf_ffn *f) { return (f->n + fused_grid() - 1) / fused_grid(); }
 
 // Ring slots that fit the shared-memory budget (0 if fewer than two).
-int fused_slots(const asf_ffn *f, int NB) {
+int fused_slots(const asf_ffn *f, int NB, int mask_words) {
   const int M = f->act == ASF_ACT_REGLU ? 3 : 2;
   for (int ns = 16; ns >= 2; --ns)
-    if (fused_layout(ns, f->d, M, esize(f->wdtype), NB, fused_nl_max(f)).total <= fused_smem_budget()) return ns;
+    if (fused_layout(ns, f->d, M, esize(f->wdtype), NB, fused_nl_max(f), mask_words).total <= fused_smem_budget())
+      return ns;
   return 0;
 }
 
@@ -1668,69 +1663,89 @@ bool fused_ok(const asf_ffn *f, int B) {
   const int nb = fused_nb(B), q = fused_maxq(f);
   if (!nb || !q) return false;
   if (q * vec_of(f->wdtype) * nb > 64) return false;   // y accumulators per lane
-  return fused_slots(f, nb) >= 2;
+  return fused_slots(f, nb, 0) >= 2;
 }
+
+// The union mask the fused kernel ranks itself (combined predict + FFN call);
+// mask == nullptr: the list comes from idx/count.
+struct MaskList {
+  const uint32_t *mask = nullptr;
+  int n_words = 0;
+  int32_t *idx_out = nullptr;
+  int32_t *count_out = nullptr;
+};
 
 template <typename T, int NB, int MAXQ, bool REGLU>
 cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
-                        float *y, Header *hdr, cudaStream_t st) {
+                        float *y, Header *hdr, cudaStream_t st, const MaskList &ml) {
   if constexpr (MAXQ * Vec<T>::N * NB > 64) {
     return cudaErrorInvalidConfiguration;
   } else {
     const int M = REGLU ? 3 : 2;
-    const int NS = fused_slots(f, NB);
-    const FusedLayout L = fused_layout(NS, f->d, M, (int)sizeof(T), NB, fused_nl_max(f));
+    const int mw = ml.mask ? ml.n_words : 0;
+    const int NS = fused_slots(f, NB, mw);
+    const FusedLayout L = fused_layout(NS, f->d, M, (int)sizeof(T), NB, fused_nl_max(f), mw);
     const int threads = (kFusedWarps + 1) * kWarp;
     auto kern = k_sparse_ffn<T, NB, MAXQ, REGLU>;
     const int G = fused_grid();
     cudaError_t e = launch(kern, dim3(G), dim3(threads), L.total, st, (const T *)f->Wg, (const T *)f->Wu,
-                           (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count, NS,
-                           idx ? std::max(0, f->hot_rows) : 0, ffn_rs(f), ffn_packed(f) ? 1 : 0, part, y, hdr);
+                           (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count, ml.mask,
+                           ml.n_words, ml.idx_out, ml.count_out, NS,
+                           (idx || ml.mask) ? std::max(0, f->hot_rows) : 0, ffn_rs(f), ffn_packed(f) ? 1 : 0, part,
+                           y, hdr, l2_next_of(f));
     if (e != cudaSuccess) return e;
     return launch(k_reduce_partials, dim3((f->d + kWarp - 1) / kWarp, B), dim3(kReduceWarps * kWarp), 0, st,
-                  (const float *)part, G, B, f->d, y, l2_next_of(f));
+                  (const float *)part, G, B, f->d, y);
   }
 }
 
 template <typename T, int NB, int MAXQ>
 cudaError_t run_fused_a(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
-                        float *y, Header *hdr, cudaStream_t st) {
-  if (f->act == ASF_ACT_REGLU) return run_fused_k<T, NB, MAXQ, true>(f, x, B, idx, count, part, y, hdr, st);
-  return run_fused_k<T, NB, MAXQ, false>(f, x, B, idx, count, part, y, hdr, st);
+                        float *y, Header *hdr, cudaStream_t st, const MaskList &ml) {
+  if (f->act == ASF_ACT_REGLU) return run_fused_k<T, NB, MAXQ, true>(f, x, B, idx, count, part, y, hdr, st, ml);
+  return run_fused_k<T, NB, MAXQ, false>(f, x, B, idx, count, part, y, hdr, st, ml);
 }
 
 template <typename T, int NB>
 cudaError_t run_fused_q(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
-                        float *y, Header *hdr, cudaStream_t st) {
+                        float *y, Header *hdr, cudaStream_t st, const MaskList &ml) {
   switch (fused_maxq(f)) {
-    case 1: return run_fused_a<T, NB, 1>(f, x, B, idx, count, part, y, hdr, st);
-    case 2: return run_fused_a<T, NB, 2>(f, x, B, idx, count, part, y, hdr, st);
-    case 4: return run_fused_a<T, NB, 4>(f, x, B, idx, count, part, y, hdr, st);
-    default: return run_fused_a<T, NB, 6>(f, x, B, idx, count, part, y, hdr, st);
+    case 1: return run_fused_a<T, NB, 1>(f, x, B, idx, count, part, y, hdr, st, ml);
+    case 2: return run_fused_a<T, NB, 2>(f, x, B, idx, count, part, y, hdr, st, ml);
+    case 4: return run_fused_a<T, NB, 4>(f, x, B, idx, count, part, y, hdr, st, ml);
+    default: return run_fused_a<T, NB, 6>(f, x, B, idx, count, part, y, hdr, st, ml);
   }
 }
 
 template <typename T>
 cudaError_t run_fused(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
-                      float *y, Header *hdr, cudaStream_t st) {
+                      float *y, Header *hdr, cudaStream_t st, const MaskList &ml) {
   switch (fused_nb(B)) {
-    case 1: return run_fused_q<T, 1>(f, x, B, idx, count, part, y, hdr, st);
-    case 2: return run_fused_q<T, 2>(f, x, B, idx, count, part, y, hdr, st);
-    default: return run_fused_q<T, 4>(f, x, B, idx, count, part, y, hdr, st);
+    case 1: return run_fused_q<T, 1>(f, x, B, idx, count, part, y, hdr, st, ml);
+    case 2: return run_fused_q<T, 2>(f, x, B, idx, count, part, y, hdr, st, ml);
+    default: return run_fused_q<T, 4>(f, x, B, idx, count, part, y, hdr, st, ml);
   }
 }
 
+// The fused kernel can rank the predictor's mask itself: the mask's words
+// still leave at least two ring slots.
+bool fused_mask_ok(const asf_ffn *f, int B) {
+  if (!fused_ok(f, B) || !fused_enabled()) return false;
+  return fused_slots(f, fused_nb(B), n_words_of(f->n)) >= 2;
+}
+
+// Sparse (idx != NULL), dense (idx == NULL) or mask-ranked (ml.mask) FFN.
+// hdr: the workspace header; scratch: this call's part of the workspace.
 template <typename T>
 asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *y,
-                 void *ws, cudaStream_t st) {
-  unsigned char *base = static_cast<unsigned char *>(ws);
-  Header *hdr = reinterpret_cast<Header *>(base);
-  float *a = reinterpret_cast<float *>(base + kHeaderBytes);
-  float *part = reinterpret_cast<float *>(base + kHeaderBytes + r256((size_t)f->n * B * 4));
+                 Header *hdr, unsigned char *scratch, cudaStream_t st, const MaskList &ml = MaskList()) {
+  float *a = reinterpret_cast<float *>(scratch);
+  float *part = reinterpret_cast<float *>(scratch + r256((size_t)f->n * B * 4));
   if (fused_ok(f, B) && fused_enabled()) {
-    float *cpart = reinterpret_cast<float *>(base + kHeaderBytes);
-    return cuda_status(run_fused<T>(f, x, B, idx, count, cpart, y, hdr, st));
+    float *cpart = reinterpret_cast<float *>(scratch);
+    return cuda_status(run_fused<T>(f, x, B, idx, count, cpart, y, hdr, st, ml));
   }
+  if (ml.mask) return ASF_ERR_UNSUPPORTED;   // callers check fused_mask_ok first
   const int nbg = pick_nb(B, (size_t)f->d * sizeof(T));
   cudaError_t e;
   switch (nbg) {
@@ -1748,6 +1763,33 @@ asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, con
     default: e = run_down<T, 8>(f, B, idx, count, a, part, y, hdr, st); break;
   }
   return cuda_status(e);
+}
+
+// One layer, predictor then sparse FFN.  Workspace: header | predictor
+// scratch (mask, h) | FFN scratch.  When layer 2 leaves the union mask and the
+// fused FFN can rank it, no compaction kernel runs: the FFN kernel builds its
+// own part of the list from the mask and writes idx/count on the way.
+template <typename T>
+asf_status predict_ffn_t(const asf_predictor *p, const asf_ffn *f, const void *x, int B, float thr, int32_t *idx,
+                         int32_t *count, float *y, void *ws, cudaStream_t st) {
+  unsigned char *base = static_cast<unsigned char *>(ws);
+  Header *hdr = reinterpret_cast<Header *>(base);
+  uint32_t *mask = reinterpret_cast<uint32_t *>(base + kHeaderBytes);
+  float *h = reinterpret_cast<float *>(base + kHeaderBytes + mask_region(p));
+  unsigned char *fs = base + kHeaderBytes + pred_scratch(p, B);
+  bool mask_only = false;
+  cudaError_t e = predict_layers<T>(p, x, B, thr, idx, count, hdr, mask, h, st, mask_only);
+  if (e != cudaSuccess) return ASF_ERR_CUDA;
+  if (mask_only && fused_mask_ok(f, B)) {
+    MaskList ml;
+    ml.mask = mask;
+    ml.n_words = n_words_of(p->n);
+    ml.idx_out = idx;
+    ml.count_out = count;
+    return ffn_t<T>(f, x, B, nullptr, nullptr, y, hdr, fs, st, ml);
+  }
+  if (mask_only && launch_compact(p, mask, idx, count, st) != cudaSuccess) return ASF_ERR_CUDA;
+  return ffn_t<T>(f, x, B, idx, count, y, hdr, fs, st);
 }
 
 template <typename T>
@@ -1801,7 +1843,7 @@ asf_status noalloc_scratch(void **out) {
 // ======================================================================== //
 extern "C" {
 
-int32_t asf_version(void) { return 103; }
+int32_t asf_version(void) { return 104; }
 
 const char *asf_status_string(asf_status s) {
   switch (s) {
@@ -1821,14 +1863,11 @@ size_t asf_workspace_bytes(const asf_predictor *pred, const asf_ffn *ffn, int32_
   if (max_batch < 1 || max_batch > ASF_MAX_BATCH) return 0;
   if (!pred && !ffn) return 0;
   size_t need = 0;
-  if (pred) {
-    if (check_pred(pred) != ASF_OK) return 0;
-    need = std::max(need, pred_scratch(pred, max_batch));
-  }
-  if (ffn) {
-    if (check_ffn(ffn) != ASF_OK) return 0;
-    need = std::max(need, ffn_scratch(ffn, max_batch));
-  }
+  if (pred && check_pred(pred) != ASF_OK) return 0;
+  if (ffn && check_ffn(ffn) != ASF_OK) return 0;
+  // both: room for the combined call, whose FFN scratch follows the predictor's
+  if (pred) need += pred_scratch(pred, max_batch);
+  if (ffn) need += ffn_scratch(ffn, max_batch);
   return kHeaderBytes + need;
 }
 
@@ -1863,8 +1902,30 @@ asf_status asf_sparse_ffn(const asf_ffn *ffn, const void *x, int32_t B, const in
   if (!al16(x) || !al16(y) || !al4(idx) || !al4(count)) return ASF_ERR_MISALIGNED;
   s = check_ws(ws, ws_bytes, kHeaderBytes + ffn_scratch(ffn, B));
   if (s != ASF_OK) return s;
-  if (ffn->wdtype == ASF_F16) return ffn_t<__half>(ffn, x, B, idx, count, y, ws, (cudaStream_t)stream);
-  return ffn_t<float>(ffn, x, B, idx, count, y, ws, (cudaStream_t)stream);
+  Header *hdr = static_cast<Header *>(ws);
+  unsigned char *scratch = static_cast<unsigned char *>(ws) + kHeaderBytes;
+  if (ffn->wdtype == ASF_F16) return ffn_t<__half>(ffn, x, B, idx, count, y, hdr, scratch, (cudaStream_t)stream);
+  return ffn_t<float>(ffn, x, B, idx, count, y, hdr, scratch, (cudaStream_t)stream);
+}
+
+asf_status asf_predict_sparse_ffn(const asf_predictor *pred, const asf_ffn *ffn, const void *x, int32_t B,
+                                  float tau, int32_t *idx, int32_t *count, float *y, void *ws, size_t ws_bytes,
+                                  asf_stream_t stream) {
+  asf_status s = check_pred(pred);
+  if (s != ASF_OK) return s;
+  s = check_ffn(ffn);
+  if (s != ASF_OK) return s;
+  if (pred->d != ffn->d || pred->n != ffn->n || pred->wdtype != ffn->wdtype) return ASF_ERR_INVALID_ARG;
+  if (!x || !idx || !count || !y) return ASF_ERR_INVALID_ARG;
+  if (B < 1 || B > ASF_MAX_BATCH) return ASF_ERR_INVALID_ARG;
+  if (!(tau > 0.f && tau < 1.f)) return ASF_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(y) || !al4(idx) || !al4(count)) return ASF_ERR_MISALIGNED;
+  s = check_ws(ws, ws_bytes, kHeaderBytes + pred_scratch(pred, B) + ffn_scratch(ffn, B));
+  if (s != ASF_OK) return s;
+  const float thr = (float)std::log((double)tau / (1.0 - (double)tau));
+  if (pred->wdtype == ASF_F16)
+    return predict_ffn_t<__half>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream);
+  return predict_ffn_t<float>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream);
 }
 
 asf_status asf_dense_ffn(const asf_ffn *ffn, const void *x, int32_t B, float *y, void *ws, size_t ws_bytes,
@@ -1876,8 +1937,10 @@ asf_status asf_dense_ffn(const asf_ffn *ffn, const void *x, int32_t B, float *y,
   if (!al16(x) || !al16(y)) return ASF_ERR_MISALIGNED;
   s = check_ws(ws, ws_bytes, kHeaderBytes + ffn_scratch(ffn, B));
   if (s != ASF_OK) return s;
-  if (ffn->wdtype == ASF_F16) return ffn_t<__half>(ffn, x, B, nullptr, nullptr, y, ws, (cudaStream_t)stream);
-  return ffn_t<float>(ffn, x, B, nullptr, nullptr, y, ws, (cudaStream_t)stream);
+  Header *hdr = static_cast<Header *>(ws);
+  unsigned char *scratch = static_cast<unsigned char *>(ws) + kHeaderBytes;
+  if (ffn->wdtype == ASF_F16) return ffn_t<__half>(ffn, x, B, nullptr, nullptr, y, hdr, scratch, (cudaStream_t)stream);
+  return ffn_t<float>(ffn, x, B, nullptr, nullptr, y, hdr, scratch, (cudaStream_t)stream);
 }
 
 asf_status asf_activation_counts(const asf_ffn *ffn, const void *x, int32_t T, int64_t *counts, void *ws,
@@ -1960,8 +2023,10 @@ asf_status asf_sparse_ffn_noalloc(const asf_ffn *ffn, const void *x, int32_t B, 
   cudaStream_t st = (cudaStream_t)stream;
   // counters and the fault word must start at zero; the rest is overwritten
   if (cudaMemsetAsync(ws, 0, kHeaderBytes, st) != cudaSuccess) return ASF_ERR_CUDA;
-  s = ffn->wdtype == ASF_F16 ? ffn_t<__half>(ffn, x, B, idx, count, y, ws, st)
-                             : ffn_t<float>(ffn, x, B, idx, count, y, ws, st);
+  Header *hdr = static_cast<Header *>(ws);
+  unsigned char *scratch = static_cast<unsigned char *>(ws) + kHeaderBytes;
+  s = ffn->wdtype == ASF_F16 ? ffn_t<__half>(ffn, x, B, idx, count, y, hdr, scratch, st)
+                             : ffn_t<float>(ffn, x, B, idx, count, y, hdr, scratch, st);
   if (s != ASF_OK) return s;
   if (fault && cudaMemcpyAsync(fault, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return ASF_ERR_CUDA;

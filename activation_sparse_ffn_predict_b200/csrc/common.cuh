@@ -25,12 +25,21 @@ struct Header {
 static_assert(sizeof(Header) <= kHeaderBytes, "header too large");
 
 // ---------------------------------------------------------------- PTX --
-// Streaming 16-byte load of read-only weights: skip L1 allocation.
+// L2 policy for weight streams: their lines are the first evicted, so the
+// streams do not push out what every kernel re-reads -- its code, and the
+// small per-step data (x, h, the union mask, index lists, partial sums).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// Streaming 16-byte load of read-only weights: skip L1, evict first from L2.
 __device__ __forceinline__ uint4 ld_stream(const void *p) {
   uint4 v;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-      : "l"(p));
+      : "l"(p), "l"(l2_evict_first()));
   return v;
 }
 
@@ -113,9 +122,27 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
+// The same for weight streams, with the L2 evict-first policy (pol from
+// l2_evict_first()).
+__device__ __forceinline__ void bulk_g2s_stream(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                                uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
 // Named barrier over the first `threads` threads of the CTA.
 __device__ __forceinline__ void named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Producer side of a named barrier: marks arrival without waiting; the
+// threads that bar.sync on the same id (count includes the arrivers) see this
+// thread's earlier memory accesses once they pass it.
+__device__ __forceinline__ void named_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Ticket for "last CTA to finish" patterns: callers __syncthreads() first so

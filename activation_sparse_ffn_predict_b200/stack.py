@@ -1,8 +1,9 @@
 """A decode step over a stack of FFN layers: predictor then sparse FFN per layer.
 
-One step takes the B tokens' FFN inputs for every layer (``x[l]``), runs
-asf_predict and asf_sparse_ffn for l = 0..L-1 in order on one stream, and
-leaves y[l], idx[l], count[l] on the device.  The launch sequence is captured
+One step takes the B tokens' FFN inputs for every layer (``x[l]``), runs the
+predictor and the sparse FFN (one asf_predict_sparse_ffn call) for
+l = 0..L-1 in order on one stream, and leaves y[l], idx[l], count[l] on the
+device.  The launch sequence is captured
 once into a CUDA graph; kernels inside it overlap through programmatic
 dependent launch (each waits for its predecessor before reading its inputs).
 """
@@ -12,14 +13,17 @@ from typing import List, Optional, Sequence
 
 import torch
 
-from .api import (FFN, Predictor, Workspace, asf_dense_ffn, asf_predict, asf_sparse_ffn)
+from .api import (FFN, Predictor, Workspace, asf_dense_ffn, asf_predict, asf_predict_sparse_ffn,
+                  asf_sparse_ffn)
 
 
 class LayerStack:
     def __init__(self, preds: Sequence[Optional[Predictor]], ffns: Sequence[FFN], batch: int,
-                 tau: float = 0.5, mode: str = "predict", device=None):
+                 tau: float = 0.5, mode: str = "predict", device=None, combined: bool = True):
         """mode: "predict" (predictor + sparse FFN), "sparse" (sparse FFN over
-        caller-filled idx/count), or "dense" (all neurons)."""
+        caller-filled idx/count), or "dense" (all neurons).  combined: in
+        predict mode, one asf_predict_sparse_ffn call per layer instead of
+        asf_predict followed by asf_sparse_ffn (same results)."""
         if mode not in ("predict", "sparse", "dense"):
             raise ValueError("mode must be predict, sparse or dense")
         self.preds = list(preds)
@@ -28,6 +32,7 @@ class LayerStack:
         self.B = int(batch)
         self.tau = float(tau)
         self.mode = mode
+        self.combined = bool(combined)
         f0 = self.ffns[0]
         dev = device if device is not None else f0.tensors[1].device
         self.d, self.n, self.dtype = f0.d, f0.n, f0.dtype
@@ -40,11 +45,19 @@ class LayerStack:
         self.graph: Optional[torch.cuda.CUDAGraph] = None
 
     def launches_per_step(self) -> int:
-        """Kernels this library launches per step: the predictor is two GEMV
-        kernels plus the compaction kernel for batches of up to 8 tokens (two
-        kernels otherwise); the sparse or dense FFN is two kernels."""
-        pred = (3 if self.B <= 8 else 2) if self.mode == "predict" else 0
-        return self.L * (pred + 2)
+        """Kernels this library launches per step, following its dispatch: the
+        predictor is two GEMV kernels plus the compaction kernel for batches
+        of up to 8 tokens (the register-streaming layer-2 kernel compacts
+        itself above that); the sparse or dense FFN is two kernels.  In the
+        combined call the fused sparse FFN (batches up to 4 whose per-lane
+        accumulators fit) ranks the mask itself and no compaction runs."""
+        if self.mode != "predict":
+            return self.L * 2
+        if self.B > 8:
+            return self.L * 4
+        if self.combined and _fused_sparse_ffn(self.d, self.dtype, self.B):
+            return self.L * 4
+        return self.L * 5
 
     def enqueue(self, stream=None) -> None:
         for l in range(self.L):
@@ -53,6 +66,10 @@ class LayerStack:
                 asf_dense_ffn(self.ffns[l], x, y, self.ws, stream)
                 continue
             cnt = self.count[l:l + 1]
+            if self.mode == "predict" and self.combined:
+                asf_predict_sparse_ffn(self.preds[l], self.ffns[l], x, self.tau, self.idx[l], cnt, y, self.ws,
+                                       stream)
+                continue
             if self.mode == "predict":
                 asf_predict(self.preds[l], x, self.tau, self.idx[l], cnt, self.ws, stream)
             asf_sparse_ffn(self.ffns[l], x, self.idx[l], cnt, y, self.ws, stream)
@@ -65,11 +82,36 @@ class LayerStack:
                 self.enqueue()
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)     # keeps the node list readable
         with torch.cuda.graph(g):
             self.enqueue()
+        g.instantiate()
         torch.cuda.synchronize()
         self.graph = g
+
+    def kernel_nodes(self) -> Optional[int]:
+        """Kernel launches recorded in the captured graph (None if the CUDA
+        runtime bindings cannot read it): the measured counterpart of
+        launches_per_step()."""
+        if self.graph is None:
+            return None
+        try:
+            from cuda.bindings import runtime as rt
+            graph = rt.cudaGraph_t(init_value=self.graph.raw_cuda_graph())
+            err, _, num = rt.cudaGraphGetNodes(graph, 0)
+            if err != rt.cudaError_t.cudaSuccess:
+                return None
+            err, nodes, num = rt.cudaGraphGetNodes(graph, num)
+            if err != rt.cudaError_t.cudaSuccess:
+                return None
+            kernels = 0
+            for nd in nodes[:num]:
+                err, kind = rt.cudaGraphNodeGetType(nd)
+                if err == rt.cudaError_t.cudaSuccess and kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                    kernels += 1
+            return kernels
+        except Exception:
+            return None
 
     def step(self) -> None:
         if self.graph is None:
@@ -81,8 +123,22 @@ class LayerStack:
         self.graph = None
 
 
+def _fused_sparse_ffn(d: int, dtype, B: int) -> bool:
+    """Whether the library runs the one-kernel sparse FFN for this shape: up to
+    4 tokens, and at most 64 fp32 accumulators per lane (d / (8 warps x 32
+    lanes x elements per 16 bytes), rounded up to 1, 2, 4 or 6 chunks, times
+    elements per chunk times the token group)."""
+    if B > 4:
+        return False
+    v = 8 if dtype == torch.float16 else 4
+    q = -(-(d // v) // 256)
+    q = next((c for c in (1, 2, 4, 6) if q <= c), None)
+    nb = next(c for c in (1, 2, 4) if B <= c)
+    return q is not None and q * v * nb <= 64
+
+
 def build_layers(weights: List, device, hot_rows: Optional[Sequence[int]] = None,
-                 l2_next: bool = False) -> tuple:
+                 l2_next: bool = True) -> tuple:
     """Predictor and FFN descriptors for a list of ``synthetic.LayerWeights`` on ``device``.
 
     hot_rows[l] (optional) is the number of leading rows of layer l that the

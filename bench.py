@@ -47,8 +47,8 @@ def parse_args(argv=None):
                    help="FFN weight layout: neuron-major packed rows, or separate W_gate/W_up/W_down^T")
     p.add_argument("--no-hot-prefetch", action="store_true",
                    help="do not pass the hot-row prefetch hint to the sparse FFN")
-    p.add_argument("--l2-next", action="store_true",
-                   help="let each sparse FFN prefetch the next layer's predictor weights into L2")
+    p.add_argument("--no-l2-next", action="store_true",
+                   help="do not let each sparse FFN prefetch the next layer's predictor weights into L2")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=1024)
@@ -247,7 +247,7 @@ def workload_config(cfg, args):
             "weights": cfg.dtype, "accumulate": "f32",
             "l2": "inputs larger than L2: every step streams rows of all layers of a stack "
                   "whose weights exceed the 126 MB L2 many times over",
-            "l2_next": (args.mode == "predict" and args.l2_next),
+            "l2_next": (args.mode == "predict" and not args.no_l2_next),
             "parallelism": f"replicas x{args.gpus}"}
 
 
@@ -320,7 +320,7 @@ def run_ours(args, cfg):
     T = args.tokens if args.tokens > 0 else cfg.tokens
     hot = cfg.hot_perm and not args.no_hot_perm
     # each layer's sparse FFN pulls the next layer's predictor weights into L2
-    l2_next = args.mode == "predict" and args.l2_next
+    l2_next = args.mode == "predict" and not args.no_l2_next
     weights, shares, hot_rows = [], [], []
     for l in range(L):
         w = S.layer_weights(cfg, l, device=device)
@@ -364,6 +364,12 @@ def run_ours(args, cfg):
         del pst
 
     st.capture()
+    # kernels per step: read from the captured graph (the stack's own mirror of
+    # the library's dispatch is the fallback)
+    launches = st.kernel_nodes()
+    launches_source = "kernel nodes of the captured CUDA graph"
+    if launches is None:
+        launches, launches_source = st.launches_per_step(), "library dispatch rules (graph not readable)"
 
     def step(i):
         t = i % T
@@ -516,7 +522,8 @@ def run_ours(args, cfg):
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": int(L * B * cfg.d * s),
                 "d2h_bytes_per_step": int(L * B * cfg.d * 4)},
-        "gpu_launches": int(args.steps * st.launches_per_step()),
+        "gpu_launches": int(args.steps * launches),
+        "gpu_launches_source": launches_source,
         "clocks": clocks,
         "step_gbs": (ffn_bytes_step + pred_bytes_step) / (step_ms * 1e-3) / 1e9,
         "touched_bytes_per_step": ffn_bytes_step + pred_bytes_step,

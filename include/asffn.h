@@ -115,7 +115,9 @@ typedef struct {
 
 /* Bytes of device workspace needed by asf_predict / asf_sparse_ffn /
  * asf_dense_ffn / asf_activation_counts for batches up to max_batch.  Either
- * descriptor may be NULL.  Returns 0 on invalid arguments. */
+ * descriptor may be NULL; with both, the size also serves
+ * asf_predict_sparse_ffn (the two scratch areas side by side).  Returns 0 on
+ * invalid arguments. */
 ASF_API size_t asf_workspace_bytes(const asf_predictor *pred, const asf_ffn *ffn, int32_t max_batch);
 
 /* Zero a freshly allocated workspace (256-byte aligned device buffer).  Must be
@@ -146,6 +148,20 @@ ASF_API asf_status asf_predict(const asf_predictor *pred, const void *x, int32_t
 ASF_API asf_status asf_sparse_ffn(const asf_ffn *ffn, const void *x, int32_t B, const int32_t *idx,
                           const int32_t *count, float *y, void *ws, size_t ws_bytes,
                           asf_stream_t stream);
+
+/* One layer of the decode path in one call: asf_predict followed by
+ * asf_sparse_ffn over the predicted list, with the same results (idx, count
+ * and y bit for bit).  For B <= 4 the sparse FFN kernel ranks the predictor's
+ * union mask itself, so no separate compaction kernel or index-list round
+ * trip sits between the two; larger batches run the two calls' kernels.
+ *   pred, ffn   descriptors of the same layer: equal d, n and wdtype
+ *   x, B, tau   as for asf_predict
+ *   idx, count  outputs as for asf_predict (the list the FFN used)
+ *   y           output as for asf_sparse_ffn
+ *   ws          at least asf_workspace_bytes(pred, ffn, B) bytes */
+ASF_API asf_status asf_predict_sparse_ffn(const asf_predictor *pred, const asf_ffn *ffn, const void *x,
+                                          int32_t B, float tau, int32_t *idx, int32_t *count, float *y,
+                                          void *ws, size_t ws_bytes, asf_stream_t stream);
 
 /* Dense FFN over all n neurons (the unsparsified reference, same kernels with an
  * implicit identity index list).  Arguments as asf_sparse_ffn. */
@@ -213,7 +229,7 @@ ASF_API asf_status asf_read_error(void *ws, int32_t *host_out, asf_stream_t stre
 ASF_API const char *asf_status_string(asf_status s);
 
 /* ABI version: major * 100 + minor (1.02: asf_ffn.hot_rows, asf_ffn.row_stride, asf_gather_rows;
- * 1.03: asf_ffn.l2_next). */
+ * 1.03: asf_ffn.l2_next; 1.04: asf_predict_sparse_ffn). */
 ASF_API int32_t asf_version(void);
 
 #ifdef __cplusplus

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.asf_version() == 103
+    assert lib.asf_version() == 104
     for code in range(8):
         assert lib.asf_status_string(code).decode() not in ("", "unknown status")
     assert lib.asf_status_string(99).decode() == "unknown status"
@@ -94,7 +94,9 @@ def test_workspace_bytes(lib):
     both = lib.asf_workspace_bytes(ctypes.byref(p), ctypes.byref(f), 4)
     assert wp >= 4096 + 100 // 32 * 4 + 32 * 4
     assert wf >= 4096 + 100 * 4 * 4
-    assert both == max(wp, wf, lib.asf_workspace_bytes(ctypes.byref(p), None, 4))
+    # with both descriptors: the predictor's and the FFN's scratch side by side
+    # (the combined call uses both at once); 4096 = the header
+    assert both == lib.asf_workspace_bytes(ctypes.byref(p), None, 4) + wf - 4096
     assert lib.asf_workspace_bytes(None, None, 1) == 0
     assert lib.asf_workspace_bytes(ctypes.byref(p), None, 0) == 0
     assert lib.asf_workspace_bytes(ctypes.byref(p), None, L.ASF_MAX_BATCH + 1) == 0
@@ -157,6 +159,34 @@ def test_sparse_ffn_rejects_bad_arguments(lib):
     assert _sparse(lib, hinted) == L.ASF_ERR_INVALID_ARG
     assert lib.asf_dense_ffn(ctypes.byref(f), FAKE, 1, FAKE, FAKE, need - 1, None) == L.ASF_ERR_WORKSPACE
     assert lib.asf_dense_ffn(ctypes.byref(f), FAKE, 0, FAKE, FAKE, need, None) == L.ASF_ERR_INVALID_ARG
+
+
+def _combined(lib, p, f, x=FAKE, B=1, tau=0.5, idx=FAKE, cnt=FAKE, y=FAKE, ws=FAKE, wsb=None):
+    if wsb is None:
+        wsb = lib.asf_workspace_bytes(ctypes.byref(p), ctypes.byref(f), max(1, min(B, L.ASF_MAX_BATCH)))
+    return lib.asf_predict_sparse_ffn(ctypes.byref(p) if p is not None else None,
+                                      ctypes.byref(f) if f is not None else None, x, B, tau, idx, cnt, y,
+                                      ws, wsb, None)
+
+
+def test_combined_call_rejects_bad_arguments(lib):
+    p, f = _pred(), _ffn()
+    assert _combined(lib, None, f, wsb=1 << 30) == L.ASF_ERR_INVALID_ARG
+    assert _combined(lib, p, None, wsb=1 << 30) == L.ASF_ERR_INVALID_ARG
+    assert _combined(lib, _pred(d=64), _ffn(d=72), wsb=1 << 30) == L.ASF_ERR_INVALID_ARG   # d differs
+    assert _combined(lib, _pred(n=100), _ffn(n=101), wsb=1 << 30) == L.ASF_ERR_INVALID_ARG  # n differs
+    assert _combined(lib, _pred(dt=L.ASF_F32), _ffn(), wsb=1 << 30) == L.ASF_ERR_INVALID_ARG  # dtype differs
+    assert _combined(lib, p, f, x=0) == L.ASF_ERR_INVALID_ARG
+    assert _combined(lib, p, f, y=0) == L.ASF_ERR_INVALID_ARG
+    assert _combined(lib, p, f, B=0) == L.ASF_ERR_INVALID_ARG
+    assert _combined(lib, p, f, B=33, wsb=1 << 30) == L.ASF_ERR_INVALID_ARG
+    assert _combined(lib, p, f, tau=1.0) == L.ASF_ERR_INVALID_ARG
+    assert _combined(lib, p, f, y=FAKE + 8) == L.ASF_ERR_MISALIGNED
+    assert _combined(lib, p, f, idx=FAKE + 2) == L.ASF_ERR_MISALIGNED
+    need = lib.asf_workspace_bytes(ctypes.byref(p), ctypes.byref(f), 1)
+    assert _combined(lib, p, f, wsb=need - 1) == L.ASF_ERR_WORKSPACE
+    # the predictor-only size is not enough for the combined call
+    assert _combined(lib, p, f, wsb=lib.asf_workspace_bytes(ctypes.byref(p), None, 1)) == L.ASF_ERR_WORKSPACE
 
 
 def test_offline_calls_reject_bad_arguments(lib):

@@ -82,6 +82,37 @@ def test_predict_then_sparse_end_to_end(layer, B):
     assert rel_err(y.cpu().numpy(), ref) <= TOL[layer.cfg.dtype]
 
 
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 8, 12, 32])
+def test_combined_call_is_bitwise_the_two_calls(layer, B):
+    # asf_predict_sparse_ffn: for small batches the FFN kernel ranks the union
+    # mask itself (no compaction kernel); idx, count and y equal those of
+    # asf_predict + asf_sparse_ffn bit for bit, and match the oracle
+    rows = slice(5, 5 + B)
+    x = layer.Xd[rows].contiguous()
+    n, d = layer.cfg.n, layer.cfg.d
+    outs = []
+    for combined in (False, True):
+        idx = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+        cnt = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+        y = torch.full((B, d), float("nan"), dtype=torch.float32, device="cuda")
+        if combined:
+            A.asf_predict_sparse_ffn(layer.pred, layer.ffn, x, layer.cfg.tau, idx, cnt, y, layer.ws)
+        else:
+            A.asf_predict(layer.pred, x, layer.cfg.tau, idx, cnt, layer.ws)
+            A.asf_sparse_ffn(layer.ffn, x, idx, cnt, y, layer.ws)
+        torch.cuda.synchronize()
+        outs.append((idx.cpu().numpy(), int(cnt.item()), y.cpu().numpy()))
+    (i0, c0, y0), (i1, c1, y1) = outs
+    assert c0 == c1
+    np.testing.assert_array_equal(i0, i1)          # the list, and the untouched tail
+    assert (i1[c1:] == -7).all()
+    np.testing.assert_array_equal(y0, y1)
+    ref_idx = layer.oracle_idx(rows)
+    np.testing.assert_array_equal(i1[:c1], ref_idx)
+    assert rel_err(y1, layer.oracle_y(rows, ref_idx)) <= TOL[layer.cfg.dtype]
+    assert layer.error() == 0
+
+
 @pytest.mark.parametrize("B", [1, 5, 32])
 def test_dense_matches_oracle(layer, B):
     rows = slice(0, B)

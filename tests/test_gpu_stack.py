@@ -15,10 +15,11 @@ from activation_sparse_ffn_predict_b200.stack import LayerStack, build_layers
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,mode,l2_next", [(1, "predict", False), (4, "predict", False),
-                                            (1, "dense", False), (4, "dense", False),
-                                            (1, "predict", True), (12, "predict", True)])
-def test_graph_stack_matches_oracle(B, mode, l2_next):
+@pytest.mark.parametrize("B,mode,l2_next,combined", [
+    (1, "predict", False, True), (4, "predict", False, True), (1, "predict", False, False),
+    (6, "predict", False, True), (1, "dense", False, True), (4, "dense", False, True),
+    (1, "predict", True, True), (12, "predict", True, True)])
+def test_graph_stack_matches_oracle(B, mode, l2_next, combined):
     ensure_built()
     cfg = S.get("llama2_7b_reglu").with_(d=1024, n=2752, r=128, layers=3)
     tokens = 3 * B
@@ -33,8 +34,10 @@ def test_graph_stack_matches_oracle(B, mode, l2_next):
         devs.append(w.to("cuda"))
         xs.append(X)
     preds, ffns = build_layers(devs, "cuda", l2_next=l2_next)
-    st = LayerStack(preds, ffns, B, cfg.tau, mode=mode)
+    st = LayerStack(preds, ffns, B, cfg.tau, mode=mode, combined=combined)
     st.capture()
+    # the launch count the benchmark reports is the graph's own kernel count
+    assert st.kernel_nodes() == st.launches_per_step()
     for step in range(3):
         rows = slice(step * B, step * B + B)
         for l in range(cfg.layers):

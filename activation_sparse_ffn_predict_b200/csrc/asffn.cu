@@ -46,7 +46,10 @@ constexpr int kTargetCtas = 296;      // 2 CTAs on each of the 148 SMs
 constexpr size_t kSmemBudget = 96 * 1024;
 constexpr int kFusedWarps = 8;        // consumer warps of the fused sparse FFN
 constexpr int kMaxGrid = 256;         // upper bound of one-CTA-per-SM grids (partials, counts)
-constexpr size_t kFusedSmemDefault = 140 * 1024;
+// Shared memory of the sparse FFN's ring: deep enough to keep ~8 neurons'
+// rows in flight per SM, while the layer-1 predictor kernel (one token group
+// of x) still fits beside it, so the next layer can start under its tail.
+constexpr size_t kFusedSmemDefault = 200 * 1024;
 constexpr uint64_t kWaitNs = 200ull * 1000 * 1000;  // bound on any mbarrier wait
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }

@@ -45,8 +45,9 @@ def parse_args(argv=None):
     p.add_argument("--no-hot-perm", action="store_true", help="keep neuron id order")
     p.add_argument("--layout", choices=["packed", "split"], default="packed",
                    help="FFN weight layout: neuron-major packed rows, or separate W_gate/W_up/W_down^T")
-    p.add_argument("--no-hot-prefetch", action="store_true",
-                   help="do not pass the hot-row prefetch hint to the sparse FFN")
+    p.add_argument("--hot-prefetch", action="store_true",
+                   help="pass the hot-row prefetch hint to the sparse FFN (off by default: the rows it "
+                        "warms that the list then skips cost more than the warm-up saves)")
     p.add_argument("--no-l2-next", action="store_true",
                    help="do not let each sparse FFN prefetch the next layer's predictor weights into L2")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -103,6 +104,18 @@ def traffic_record(kernel_key: str):
     if rec.get("source_sha") != source_sha():
         return None
     return rec.get("kernels", {}).get(kernel_key)
+
+
+def traffic_per_launch(rec, algorithmic_bytes: float):
+    """DRAM bytes per launch of the dominant kernel: a captured per-launch
+    figure, or a captured ratio of DRAM bytes to algorithmic bytes applied to
+    this run's algorithmic bytes per launch (the capture ran a smaller case of
+    the same kernel, and traffic grows with the rows a launch gathers)."""
+    if not rec:
+        return None
+    if "dram_bytes_per_algorithmic_byte" in rec:
+        return float(rec["dram_bytes_per_algorithmic_byte"]) * algorithmic_bytes
+    return rec.get("dram_bytes_per_launch")
 
 
 class ClockSampler:
@@ -248,6 +261,7 @@ def workload_config(cfg, args):
             "l2": "inputs larger than L2: every step streams rows of all layers of a stack "
                   "whose weights exceed the 126 MB L2 many times over",
             "l2_next": (args.mode == "predict" and not args.no_l2_next),
+            "hot_row_hint": bool(args.hot_prefetch),
             "parallelism": f"replicas x{args.gpus}"}
 
 
@@ -327,7 +341,7 @@ def run_ours(args, cfg):
         if hot:
             w, share, hr = hot_permute_layer(cfg, l, w, device)
             shares.append(share)
-            hot_rows.append(0 if args.no_hot_prefetch else hr)
+            hot_rows.append(hr if args.hot_prefetch else 0)
         weights.append(w)
     if args.layout == "packed":
         # neuron-major packed rows: one bulk copy per neuron in the sparse FFN
@@ -510,7 +524,8 @@ def run_ours(args, cfg):
             "achieved": ffn_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": ffn_gbs / hbm_peak,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
             "frac_of_nominal_7700": ffn_gbs / NOMINAL_HBM_GBS,
-            "traffic": (tr["dram_bytes_per_launch"] if tr else None),
+            "traffic": traffic_per_launch(tr, ffn_bytes_prof / (nprof * L)),
+            "traffic_source": (tr or {}).get("source"),
             "algorithmic_bytes_per_launch": ffn_bytes_prof / (nprof * L),
             "launch_ms": ffn_call_ms}
     line = {
@@ -528,6 +543,9 @@ def run_ours(args, cfg):
         "step_gbs": (ffn_bytes_step + pred_bytes_step) / (step_ms * 1e-3) / 1e9,
         "touched_bytes_per_step": ffn_bytes_step + pred_bytes_step,
         "active_per_layer_mean": float(counts[tok_seq].mean()),
+        # small profiling runs: every (token, layer) list length, to set the
+        # algorithmic bytes of individual captured launches beside their traffic
+        **({"active_counts": counts.tolist()} if counts.size <= 64 else {}),
         "predictor_call": ({"ms": pred_call_ms, "gbs": pred_gbs, "frac": pred_gbs / hbm_peak,
                             "bytes": pred_bytes_l} if pred_gbs else None),
         "hot_share_top20": (float(np.mean(shares)) if shares else None),

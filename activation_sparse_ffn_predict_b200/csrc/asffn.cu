@@ -212,16 +212,56 @@ __global__ void __launch_bounds__(kThreads)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row0 = blockIdx.x * rpc;
   const int row1 = min(r, row0 + rpc);
-  // No L2 prefetch here: this grid becomes resident while the previous
-  // layer's sparse FFN starts its row stream, and weight traffic issued now
-  // would delay those rows (the asf_ffn.l2_next hint prefetches the weights
-  // once the rows are queued).  The next kernel reads only weights before it
-  // waits on this one.
+  const int nvec = d / V;
+  // One row per warp and one token group: the warp's W1 row goes into
+  // registers before the wait.  This grid becomes resident as the previous
+  // layer's sparse FFN starts, while that kernel ranks its list and HBM is
+  // idle; a row (8 KB at d = 4096) fits that window.  (Prefetching more --
+  // this layer's W2 as well -- spilled into the FFN's row stream and delayed
+  // it.)  The next kernel reads only weights before it waits on this one.
+  const bool early = U * kWarp >= nvec && row1 - row0 <= kWarps && B <= NB;
+  const int erow = row0 + warp;
+  uint4 wpre[U];
+  float bias_pre = 0.f;
+  if (early) {
+    if (erow < row1) bias_pre = __ldg(b1 + erow);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = lane + u * kWarp;
+      wpre[u] = (erow < row1 && c < nvec) ? ld_stream_early(W1 + (size_t)erow * d + (size_t)c * V)
+                                          : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   pdl_trigger();
   pdl_wait();
   for (int w = blockIdx.x * kThreads + threadIdx.x; w < n_words; w += gridDim.x * kThreads)
     mask_words[w] = 0u;
-  const int nvec = d / V;
+  if (early) {
+    stage_tokens<T, NB>(xs, x, d, 0, B);
+    __syncthreads();
+    if (erow < row1) {
+      float acc[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+      const float bias = bias_pre;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = lane + u * kWarp;
+        if (c < nvec) {
+#pragma unroll
+          for (int b = 0; b < NB; ++b)
+            acc[b] = Vec<T>::dot(wpre[u], *reinterpret_cast<const uint4 *>(xs + (size_t)b * d + (size_t)c * V),
+                                 acc[b]);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float sum = warp_sum(acc[b]);
+        if (lane == b && b < B) h[(size_t)b * r + erow] = fmaxf(sum + bias, 0.f);
+      }
+    }
+    return;
+  }
   for (int g0 = 0; g0 < B; g0 += NB) {
     const int nb = min(NB, B - g0);
     __syncthreads();

@@ -43,6 +43,16 @@ __device__ __forceinline__ uint4 ld_stream(const void *p) {
   return v;
 }
 
+// The same, as a volatile asm: it stays where it is written, so weights loaded
+// ahead of griddepcontrol.wait are in flight while the kernel waits.
+__device__ __forceinline__ uint4 ld_stream_early(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(l2_evict_first()));
+  return v;
+}
+
 // Load of data another kernel (or CTA) produced: served from L2, never L1.
 __device__ __forceinline__ int ld_cg_i32(const int32_t *p) { return __ldcg(p); }
 __device__ __forceinline__ float ld_cg_f32(const float *p) { return __ldcg(p); }

@@ -138,13 +138,14 @@ def _fused_sparse_ffn(d: int, dtype, B: int) -> bool:
 
 
 def build_layers(weights: List, device, hot_rows: Optional[Sequence[int]] = None,
-                 l2_next: bool = True) -> tuple:
+                 l2_next: bool = False) -> tuple:
     """Predictor and FFN descriptors for a list of ``synthetic.LayerWeights`` on ``device``.
 
     hot_rows[l] (optional) is the number of leading rows of layer l that the
     offline profile found active for most tokens (the prefetch hint).  With
     l2_next, layer l's sparse FFN prefetches the predictor weights of layer
-    l+1 (of layer 0 after the last layer: the next token's first layer) into L2."""
+    l+1 (of layer 0 after the last layer: the next token's first layer) into
+    L2; off by default, since the benchmark stack measured faster without it."""
     preds, ffns = [], []
     for l, w in enumerate(weights):
         preds.append(Predictor(w.W1, w.b1, w.W2, w.b2))

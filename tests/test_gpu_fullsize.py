@@ -95,8 +95,15 @@ def test_fullsize_predict_and_sparse_ffn(full_layer):
             y = torch.full((B, cfg.d), float("nan"), dtype=torch.float32, device="cuda")
             A.asf_predict(fl.pred, x, cfg.tau, idx, cnt, fl.ws)
             A.asf_sparse_ffn(fl.ffn, x, idx, cnt, y, fl.ws)
+            # the combined call (the benchmark's path) gives the same list and y, bit for bit
+            idx2 = torch.full((cfg.n,), -5, dtype=torch.int32, device="cuda")
+            cnt2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+            y2 = torch.full((B, cfg.d), float("nan"), dtype=torch.float32, device="cuda")
+            A.asf_predict_sparse_ffn(fl.pred, fl.ffn, x, cfg.tau, idx2, cnt2, y2, fl.ws)
             torch.cuda.synchronize()
             c = int(cnt.item())
+            assert int(cnt2.item()) == c
+            assert torch.equal(idx[:c], idx2[:c]) and torch.equal(y, y2)
             got = idx[:c].cpu().numpy()
             ref = fl.oracle_idx(rows)
             np.testing.assert_array_equal(got, ref)

@@ -150,8 +150,10 @@ ASF_API asf_status asf_sparse_ffn(const asf_ffn *ffn, const void *x, int32_t B, 
                           asf_stream_t stream);
 
 /* One layer of the decode path in one call: asf_predict followed by
- * asf_sparse_ffn over the predicted list, with the same results (idx, count
- * and y bit for bit).  For B <= 4 the sparse FFN kernel ranks the predictor's
+ * asf_sparse_ffn over the predicted list (the predictor-then-sparse-operator
+ * flow of the PowerInfer Guide, Step 2 predictor module feeding the Step 3
+ * sparse FFN, and the PowerInfer_x64 page's "Prediction and Caching"), with
+ * the same results (idx, count and y bit for bit).  For B <= 4 the sparse FFN kernel ranks the predictor's
  * union mask itself, so no separate compaction kernel or index-list round
  * trip sits between the two; larger batches run the two calls' kernels.
  *   pred, ffn   descriptors of the same layer: equal d, n and wdtype

@@ -265,10 +265,13 @@ def asf_gather_rows(src: torch.Tensor, dst: torch.Tensor, perm: Optional[torch.T
 
 def pack_layer(act: str, Wg: Optional[torch.Tensor], Wu: torch.Tensor, WdT: torch.Tensor,
                perm: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Neuron-major packed copy [n, m, d] of a layer's rows (optionally permuted)."""
+    """Neuron-major packed copy [k, m, d] of a layer's rows: row i is neuron
+    perm[i] (k = len(perm): a permutation, or a subset such as one rank's
+    neurons), or neuron i without perm (k = n)."""
     n, d = Wu.shape
     mats = [Wg, Wu, WdT] if act == "reglu" else [Wu, WdT]
-    out = torch.empty(n, len(mats), d, dtype=Wu.dtype, device=Wu.device)
+    k = int(perm.shape[0]) if perm is not None else n
+    out = torch.empty(k, len(mats), d, dtype=Wu.dtype, device=Wu.device)
     rb = d * Wu.element_size()
     for m, W in enumerate(mats):
         asf_gather_rows(W, out, perm, dst_offset=m * rb, dst_stride=len(mats) * rb, stream=stream)

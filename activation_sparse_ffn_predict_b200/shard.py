@@ -1,0 +1,108 @@
+"""Neuron-sharded layer across G GPUs (one process per GPU).
+
+The FFN's neurons are split across ranks -- the neuron partitioning that the
+PowerInfer_x64 page lists among its multi-GPU coordination modes (its
+architecture and tech-stack paragraph): rank g holds the predictor's W2/b2 rows and
+the gate/up/down rows of its own neurons, while W1/b1 (the predictor's first
+layer, over the whole input) are replicated.  Each rank predicts the activity
+of its own neurons and gathers only those rows with the same one-call layer
+(asf_predict_sparse_ffn) as the single-GPU path, giving a partial y over its
+neurons; one all-reduce (sum) of y [B, d] fp32 per layer combines the ranks.
+
+A neuron's prediction depends only on x and its own W2 row, so the union of
+the ranks' lists (mapped back to global ids) is exactly the single-GPU list,
+and the sum of the partial outputs is the single-GPU y up to the order of the
+fp32 additions.
+
+Ownership deals blocks of `block` consecutive rows round-robin, so a
+hot-first storage order (the offline permutation) spreads hot rows evenly
+instead of giving them all to rank 0.  The shards' rows are gathered once,
+offline, with the library's own row-gather kernel.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+from .api import (FFN, Predictor, Workspace, asf_gather_rows, asf_predict_sparse_ffn, pack_layer)
+
+
+def shard_rows(n: int, world: int, rank: int, block: int = 32) -> np.ndarray:
+    """Global ids (ascending, int32) of the neurons rank owns: blocks of
+    `block` consecutive rows dealt round-robin over the world's ranks."""
+    if not (0 <= rank < world) or n < 0 or block < 1:
+        raise ValueError("need 0 <= rank < world, n >= 0 and block >= 1")
+    nb = (n + block - 1) // block
+    mine = np.arange(rank, nb, world, dtype=np.int64)
+    rows = (mine[:, None] * block + np.arange(block, dtype=np.int64)[None, :]).ravel()
+    return rows[rows < n].astype(np.int32)
+
+
+def _gather_vector(v: torch.Tensor, rows: torch.Tensor) -> torch.Tensor:
+    """v[rows] for a 1-D fp32 device vector, through the library's gather kernel."""
+    out = torch.empty(rows.shape[0], dtype=v.dtype, device=v.device)
+    if rows.shape[0]:
+        asf_gather_rows(v.reshape(-1, 1), out.reshape(-1, 1), rows)
+    return out
+
+
+def _gather_matrix(W: torch.Tensor, rows: torch.Tensor) -> torch.Tensor:
+    out = torch.empty(rows.shape[0], W.shape[1], dtype=W.dtype, device=W.device)
+    if rows.shape[0]:
+        asf_gather_rows(W, out, rows)
+    return out
+
+
+class NeuronShard:
+    """One rank's part of one layer (``synthetic.LayerWeights``-like ``w`` on
+    this rank's device): the predictor over its neurons and its FFN rows in the
+    neuron-major packed layout."""
+
+    def __init__(self, w, rank: int, world: int, block: int = 32):
+        n = int(w.W2.shape[0])
+        dev = w.W2.device
+        self.rank, self.world = rank, world
+        self.rows_host = shard_rows(n, world, rank, block)
+        self.rows = torch.from_numpy(self.rows_host).to(dev)
+        if self.rows.shape[0] == 0:
+            raise ValueError("this rank owns no neurons: use fewer ranks or a smaller block")
+        self.W2 = _gather_matrix(w.W2, self.rows)
+        self.b2 = _gather_vector(w.b2, self.rows)
+        self.bias = _gather_vector(w.bias, self.rows)
+        self.packed = pack_layer(w.act, w.Wg, w.Wu, w.WdT, perm=self.rows)
+        self.pred = Predictor(w.W1, w.b1, self.W2, self.b2)
+        self.ffn = FFN.packed(w.act, self.packed, self.bias)
+        self.n_local = int(self.rows.shape[0])
+
+    def workspace(self, max_batch: int) -> Workspace:
+        return Workspace(self.pred, self.ffn, max_batch)
+
+    def global_ids(self, idx: torch.Tensor, count: int) -> torch.Tensor:
+        """This rank's active neurons as global ids (ascending: the ownership
+        map is increasing, so the local order is kept)."""
+        return self.rows.index_select(0, idx[:count].long())
+
+
+def combine_partials(y: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum the ranks' partial outputs in place (one all-reduce of y [B, d]);
+    a no-op without an initialised process group of more than one rank."""
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
+    return y
+
+
+def sharded_layer(shard: NeuronShard, x: torch.Tensor, tau: float, idx: torch.Tensor, count: torch.Tensor,
+                  y: torch.Tensor, ws: Workspace, group=None, stream=None) -> torch.Tensor:
+    """One layer on this rank: predict and gather its own neurons (idx/count
+    in local ids), then combine y over the ranks."""
+    asf_predict_sparse_ffn(shard.pred, shard.ffn, x, tau, idx, count, y, ws, stream)
+    return combine_partials(y, group)
+
+
+def merge_lists(per_rank: list) -> np.ndarray:
+    """The single-GPU list from the ranks' global-id lists (host arrays)."""
+    if not per_rank:
+        return np.zeros(0, dtype=np.int32)
+    return np.sort(np.concatenate([np.asarray(p, dtype=np.int64) for p in per_rank])).astype(np.int32)
+

@@ -1,26 +1,31 @@
 // libasffn: activation-sparse FFN decode path for B200 (sm_100a).
 //
-// Operations (see include/asffn.h for the ABI contract):
-//   predictor layer 1   h = ReLU(W1 x + b1)                 k_pred_l1
-//   predictor layer 2   z = W2 h + b2, z > logit(tau),       k_pred_l2
-//                       union over tokens, ascending compaction by the last CTA
-//   gate/up gather      a_k = ReLU(Wg[k].x + b_k) * Wu[k].x  k_ffn_gu
-//                       (or ReLU(Wu[k].x + b_k)) for k in idx
-//   down accumulate     y = sum_j a_j WdT[idx_j]             k_ffn_down
-//   profiler            counts[k] += #(ReLU input > 0)       k_act_counts
-//   row gather          dst[i] = src[perm[i]]                k_permute_rows
+// Operations (see include/asffn.h for the ABI contract) and their kernels:
+//   predictor layer 1   h = ReLU(W1 x + b1)                        k_pred_l1
+//   predictor layer 2   z = W2 h + b2, z > logit(tau), OR of the   k_pred2_ring (B <= 8),
+//                       per-token bits into the union mask          k_pred_l2 (B > 8, compacts
+//                                                                   in its last CTA)
+//   compaction          mask -> ascending idx, count               k_compact (asf_predict),
+//                                                                   or inside k_sparse_ffn
+//   sparse FFN          a_k = ReLU(Wg[k].x + b_k) * Wu[k].x        k_sparse_ffn + k_reduce_partials
+//                       (or ReLU(Wu[k].x + b_k)) for k in idx,      (B <= 4), k_ffn_gu + k_ffn_down
+//                       y = sum_k a_k WdT[k]                        (larger batches)
+//   profiler            counts[k] += #(ReLU input > 0)             k_act_counts
+//   row gather          dst[i] = src[perm[i]]                      k_permute_rows
 //
 // Method: "PowerInfer Guide: Exploiting Activation Sparsity for LLM AI" (FFN
 // equation in "The Hidden Inefficiency"; predictor equation in section 3
 // "Adaptive Online Neuron Predictors"; section 4 "Neuron-Aware Sparse GPU
 // Operators"; Step 1 profiler) and the 2-layer MLP predictor of the
 // "PowerInfer_x64" page.  The kernels are this library's own B200 design:
-// every weight byte is streamed once with 16-byte non-allocating loads, the
-// activation vector lives in shared memory, accumulation is fp32, and every
-// cross-CTA reduction is deterministic (fixed-order sums by the last CTA to
-// finish, found with an atomic ticket; no spin-waits, no float atomics).
+// weight rows reach shared memory by cp.async.bulk into mbarrier-completed
+// rings (or registers, for the register-streaming kernels) with an L2
+// evict-first policy, and each weight byte is read once; accumulation is
+// fp32; every cross-CTA reduction is a fixed-order sum (no float atomics).
 // Consecutive kernels overlap through programmatic dependent launch: each
-// kernel may prefetch its weights into L2 before waiting for its inputs.
+// kernel touches only weights before griddepcontrol.wait and triggers its
+// successor at entry.  Every wait on an mbarrier gives up after 200 ms and
+// records ASF_ERR_TIMEOUT in the workspace error word instead of hanging.
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>

@@ -18,6 +18,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -84,13 +85,24 @@ def host_cores() -> int:
     return min(n, 64)   # OpenBLAS build limit (MAX_THREADS=64)
 
 
+def _code_only(text: str) -> str:
+    """C/CUDA source without comments and blank space: what compiles."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_sha() -> str:
+    """Hash of the kernel sources' code (comments and spacing excluded), the
+    key that ties a committed ncu traffic figure to the kernels it measured."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "activation_sparse_ffn_predict_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+        if not name.endswith((".cu", ".cuh", ".h")):
+            continue
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

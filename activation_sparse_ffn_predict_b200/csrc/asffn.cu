@@ -900,61 +900,68 @@ __host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int es
   return L;
 }
 
-// The ascending list of the set bits of a union mask (n bits in n_words
-// words), as one CTA of G needs it: slist[i] = the bit at list position
-// c + i*G.  One warp.  The words are staged in shared memory (sw, 16-byte
-// aligned, n_words rounded up to 4); each lane takes a contiguous block of
-// words and, after a warp scan of the blocks' popcounts, writes every word's
-// inclusive prefix count (spre).  Then each lane takes list positions and
-// finds its word by binary search over spre and the bit within it.  Returns
-// the number of set bits.
-__device__ __forceinline__ int list_from_mask(const uint32_t *__restrict__ mask, int n_words, int n, int c, int G,
-                                              int *slist, uint32_t *sw, int *spre) {
-  constexpr int MAXU = 4;
-  const int lane = threadIdx.x & 31;
-  const int nq = (n_words + 3) / 4;               // 16-byte groups of words
+// Ranking the set bits of a union mask (n bits in n_words words) into the
+// list positions one CTA of G takes: slist[i] = the bit at position c + i*G.
+// NT threads (the consumer warps), each owning a contiguous run of at most
+// MAXW words.  First the words' loads are issued (mask_words_load), so that
+// they are in flight while x is staged; then rank_mask_block keeps the words
+// in shared memory (sw, n_words rounded up to 4), scans the runs' popcounts
+// across the block, writes every word's inclusive prefix count (spre), and
+// finds each position's word by binary search over spre and the bit within
+// it.  Leaves the list length in *s_nl and the number of set bits in *s_cnt.
+template <int NT, int MAXW>
+__device__ __forceinline__ void mask_words_load(const uint32_t *__restrict__ mask, int n_words,
+                                                uint32_t (&w)[MAXW]) {
+  const int wpt = (n_words + NT - 1) / NT;
+  const int wb = min(n_words, (int)threadIdx.x * wpt), we = min(n_words, wb + wpt);
+#pragma unroll
+  for (int u = 0; u < MAXW; ++u) w[u] = wb + u < we ? __ldcg(mask + wb + u) : 0u;
+}
+
+template <int NT, int MAXW>
+__device__ __forceinline__ void rank_mask_block(uint32_t (&w)[MAXW], int n_words, int n, int c, int G, int *slist,
+                                                uint32_t *sw, int *spre, int *s_wsum, int *s_nl, int *s_cnt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wpt = (n_words + NT - 1) / NT;
+  const int wb = min(n_words, tid * wpt), we = min(n_words, wb + wpt);
   const uint32_t tail = (n & 31) ? ((1u << (n & 31)) - 1u) : 0xffffffffu;
-  for (int q0 = 0; q0 < nq; q0 += MAXU * kWarp) {
-    uint4 v[MAXU];
+  int tot = 0;
 #pragma unroll
-    for (int u = 0; u < MAXU; ++u) {
-      const int q = q0 + u * kWarp + lane;
-      v[u] = q < nq ? __ldcg(reinterpret_cast<const uint4 *>(mask) + q) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int u = 0; u < MAXU; ++u) {
-      const int q = q0 + u * kWarp + lane;
-      if (q < nq) {
-        uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int w = 4 * q + e;
-          w4[e] = w < n_words ? (w == n_words - 1 ? (w4[e] & tail) : w4[e]) : 0u;
-        }
-        reinterpret_cast<uint4 *>(sw)[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
+  for (int u = 0; u < MAXW; ++u) {
+    const int i = wb + u;
+    if (i < we) {
+      if (i == n_words - 1) w[u] &= tail;
+      sw[i] = w[u];
+      tot += __popc(w[u]);
     }
   }
-  __syncwarp();
-  const int per = (n_words + kWarp - 1) / kWarp;
-  const int wb = min(n_words, lane * per), we = min(n_words, wb + per);
-  int tot = 0;
-  for (int w = wb; w < we; ++w) tot += __popc(sw[w]);
   int incl = tot;
 #pragma unroll
   for (int o = 1; o < kWarp; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
-  const int cnt = __shfl_sync(0xffffffffu, incl, kWarp - 1);
-  int run = incl - tot;
-  for (int w = wb; w < we; ++w) {
-    run += __popc(sw[w]);
-    spre[w] = run;
+  if (lane == kWarp - 1) s_wsum[warp] = incl;
+  named_sync(3, NT);
+  int before = 0, all = 0;
+#pragma unroll
+  for (int q = 0; q < NT / kWarp; ++q) {
+    const int v = s_wsum[q];
+    all += v;
+    if (q < warp) before += v;
   }
-  __syncwarp();
-  const int nl = cnt > c ? (cnt - 1 - c) / G + 1 : 0;
-  for (int i = lane; i < nl; i += kWarp) {
+  int run = before + incl - tot;
+#pragma unroll
+  for (int u = 0; u < MAXW; ++u) {
+    const int i = wb + u;
+    if (i < we) {
+      run += __popc(w[u]);
+      spre[i] = run;
+    }
+  }
+  named_sync(3, NT);
+  const int nl = all > c ? (all - 1 - c) / G + 1 : 0;
+  for (int i = tid; i < nl; i += NT) {
     const int p = c + G * i;
     int lo = 0, hi = n_words - 1;          // first word whose inclusive count exceeds p
     while (lo < hi) {
@@ -965,16 +972,24 @@ __device__ __forceinline__ int list_from_mask(const uint32_t *__restrict__ mask,
     for (int q = p - (lo ? spre[lo - 1] : 0); q > 0; --q) m &= m - 1u;   // drop the lower set bits
     slist[i] = lo * 32 + __ffs(m) - 1;
   }
-  return cnt;
+  if (tid == 0) {
+    *s_nl = nl;
+    *s_cnt = all;
+  }
+  named_sync(3, NT);
 }
+
+// Most mask words per consumer thread when the sparse FFN ranks the mask.
+constexpr int kRankWords = 8;
 
 // One kernel for the whole neuron-sparse FFN of B <= NB tokens.
 //
 // CTA c of a grid of G takes list positions c, c + G, c + 2G, ...: its first
 // index loads need not wait for the count.  The list comes from idx/count, or
 // (idx == NULL) is every neuron, or (mask != NULL) is built here from the
-// predictor's union mask, whose set bits this kernel ranks itself and writes
-// out as idx_out/count_out (no separate compaction kernel).  Warp
+// predictor's union mask: the consumer warps rank its set bits (block-wide
+// scan) and the producer's idle lanes write this CTA's positions out as
+// idx_out/count_out (no separate compaction kernel).  Warp
 // kFusedWarps is the producer: one lane streams, for each of its neurons k,
 // the rows Wg[k], Wu[k], WdT[k] into a ring of NS shared-memory slots with
 // cp.async.bulk, completing on the slot's "full" mbarrier.  The 8 consumer
@@ -1001,7 +1016,8 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
   constexpr int M = REGLU ? 3 : 2;
   constexpr int NW = kFusedWarps;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_fail, s_nl;
+  __shared__ int s_fail, s_nl, s_cnt;
+  __shared__ int s_wsum[kFusedWarps];
   const FusedLayout L = fused_layout(NS, d, M, (int)sizeof(T), NB, (n + (int)gridDim.x - 1) / (int)gridDim.x,
                                      mask ? n_words : 0);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);
@@ -1056,13 +1072,34 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
 #pragma unroll
       for (int b = 0; b < NB; ++b) acc[q][e][b] = 0.f;
 
-  if (warp == NW) {
+  if (mask) {
+    // ------------------------------- the list from the mask (combined call) --
+    if (warp < NW) {
+      // consumer warps rank the mask; its words load while x is staged
+      uint32_t mw[kRankWords];
+      mask_words_load<NW * kWarp, kRankWords>(mask, n_words, mw);
+      stage16<8>(reinterpret_cast<uint4 *>(xs), reinterpret_cast<const uint4 *>(x), B * nvec, NW * kWarp);
+      for (int i = B * nvec + threadIdx.x; i < NB * nvec; i += NW * kWarp)
+        reinterpret_cast<uint4 *>(xs)[i] = make_uint4(0u, 0u, 0u, 0u);
+      uint32_t *sw = reinterpret_cast<uint32_t *>(smem + L.words);
+      rank_mask_block<NW * kWarp, kRankWords>(mw, n_words, n, cta, G, slist, sw,
+                                              reinterpret_cast<int *>(sw) + (n_words + 3) / 4 * 4, s_wsum, &s_nl,
+                                              &s_cnt);
+      named_arrive(2, (NW + 1) * kWarp);     // the list is ready for the producer
+    } else {
+      named_sync(2, (NW + 1) * kWarp);
+      if (lane > 0) {
+        // this CTA's positions of the list, written out by the lanes that do
+        // not issue copies (all CTAs together write idx_out[0..count))
+        const int nlp = s_nl;
+        for (int i = lane - 1; i < nlp; i += kWarp - 1) idx_out[cta + (size_t)G * i] = slist[i];
+        if (cta == 0 && lane == 1) *count_out = s_cnt;
+      }
+    }
+  } else if (warp == NW) {
     // -------------------------------------------------- this CTA's list --
     int cnt;
-    if (mask) {
-      uint32_t *sw = reinterpret_cast<uint32_t *>(smem + L.words);
-      cnt = list_from_mask(mask, n_words, n, cta, G, slist, sw, reinterpret_cast<int *>(sw) + (n_words + 3) / 4 * 4);
-    } else if (idx) {
+    if (idx) {
       // the count and the first 32 positions are fetched together
       const int p0 = cta + G * lane;
       const int c_raw = ld_cg_i32(count);
@@ -1081,13 +1118,6 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     // hand the list to the consumers without waiting for them
     __syncwarp();
     named_arrive(2, (NW + 1) * kWarp);
-    if (mask && lane > 0) {
-      // this CTA's positions of the list, written out by the lanes that do
-      // not issue copies (all CTAs together write idx_out[0..count))
-      const int nlp = s_nl;
-      for (int i = lane - 1; i < nlp; i += kWarp - 1) idx_out[cta + (size_t)G * i] = slist[i];
-      if (cta == 0 && lane == 1) *count_out = cnt;
-    }
   } else {
     // consumers: x into shared memory while the list is being fetched
     stage16<8>(reinterpret_cast<uint4 *>(xs), reinterpret_cast<const uint4 *>(x), B * nvec, NW * kWarp);
@@ -1779,6 +1809,7 @@ cudaError_t run_fused(const asf_ffn *f, const void *x, int B, const int32_t *idx
 // still leave at least two ring slots.
 bool fused_mask_ok(const asf_ffn *f, int B) {
   if (!fused_ok(f, B) || !fused_enabled()) return false;
+  if (n_words_of(f->n) > kRankWords * kFusedWarps * kWarp) return false;   // words per ranking thread
   return fused_slots(f, fused_nb(B), n_words_of(f->n)) >= 2;
 }
 

@@ -21,7 +21,9 @@ ASF_F16 = 1
 ASF_ACT_RELU = 0
 ASF_ACT_REGLU = 1
 ASF_MAX_BATCH = 32
-ASF_NOALLOC_SCRATCH_BYTES = 8 << 20
+ASF_NOALLOC_SCRATCH_BYTES = 32 << 20
+ASF_INJECT_NONE = 0
+ASF_INJECT_WITHHOLD_FFN_COPIES = 1
 
 
 class asf_predictor(ctypes.Structure):
@@ -46,6 +48,13 @@ PROTOTYPES = {
                                c_void_p, c_size_t, c_void_p]),
     "asf_predict_sparse_ffn": (c_int, [POINTER(asf_predictor), POINTER(asf_ffn), c_void_p, c_int32, c_float,
                                        c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "asf_predict_sparse_ffn_begin": (c_int, [POINTER(asf_predictor), POINTER(asf_ffn), c_void_p, c_int32,
+                                             c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                             c_void_p]),
+    "asf_predict_sparse_ffn_end": (c_int, [POINTER(asf_predictor), POINTER(asf_ffn), c_void_p, c_int32,
+                                           c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                           c_void_p]),
+    "asf_set_fault_injection": (c_int, [c_int32]),
     "asf_dense_ffn": (c_int, [POINTER(asf_ffn), c_void_p, c_int32, c_void_p, c_void_p, c_size_t,
                               c_void_p]),
     "asf_activation_counts": (c_int, [POINTER(asf_ffn), c_void_p, c_int32, c_void_p, c_void_p,

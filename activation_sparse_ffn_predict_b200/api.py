@@ -187,6 +187,37 @@ def asf_predict_sparse_ffn(pred: Predictor, ffn: FFN, x: torch.Tensor, tau: floa
     check(st, "asf_predict_sparse_ffn")
 
 
+def _layer_call(name: str, pred: Predictor, ffn: FFN, x: torch.Tensor, tau: float, idx: torch.Tensor,
+                count: torch.Tensor, y: torch.Tensor, ws: Workspace, stream=None) -> None:
+    if x.dtype != ffn.dtype or x.dim() != 2 or x.shape[1] != ffn.d:
+        raise ValueError("x must be [B, d] in the FFN's dtype")
+    if y.shape != (x.shape[0], ffn.d):
+        raise ValueError("y must be [B, d]")
+    st = getattr(L.load(), name)(ctypes.byref(pred.desc), ctypes.byref(ffn.desc), _dev(x, "x"),
+                                 int(x.shape[0]), float(tau), _dev(idx, "idx", torch.int32),
+                                 _dev(count, "count", torch.int32), _dev(y, "y", torch.float32),
+                                 ws.ptr, ws.nbytes, _stream(stream))
+    check(st, name)
+
+
+def asf_predict_sparse_ffn_begin(pred: Predictor, ffn: FFN, x: torch.Tensor, tau: float, idx: torch.Tensor,
+                                 count: torch.Tensor, y: torch.Tensor, ws: Workspace, stream=None) -> None:
+    """First half of asf_predict_sparse_ffn (the predictor's kernels)."""
+    _layer_call("asf_predict_sparse_ffn_begin", pred, ffn, x, tau, idx, count, y, ws, stream)
+
+
+def asf_predict_sparse_ffn_end(pred: Predictor, ffn: FFN, x: torch.Tensor, tau: float, idx: torch.Tensor,
+                               count: torch.Tensor, y: torch.Tensor, ws: Workspace, stream=None) -> None:
+    """Second half of asf_predict_sparse_ffn (compaction if needed, the sparse
+    FFN); with the same arguments after _begin it completes the layer."""
+    _layer_call("asf_predict_sparse_ffn_end", pred, ffn, x, tau, idx, count, y, ws, stream)
+
+
+def asf_set_fault_injection(mode: int) -> None:
+    """Test hook for the bounded device waits (see include/asffn.h)."""
+    check(L.load().asf_set_fault_injection(int(mode)), "asf_set_fault_injection")
+
+
 def asf_sparse_ffn_noalloc(ffn: FFN, x: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
                            y: torch.Tensor, fault: Optional[torch.Tensor] = None, stream=None) -> None:
     """asf_sparse_ffn without a workspace: for callers that cannot allocate

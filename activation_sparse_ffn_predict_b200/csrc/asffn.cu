@@ -31,6 +31,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -56,6 +57,7 @@ constexpr int kMaxGrid = 256;         // upper bound of one-CTA-per-SM grids (pa
 // of x) still fits beside it, so the next layer can start under its tail.
 constexpr size_t kFusedSmemDefault = 200 * 1024;
 constexpr uint64_t kWaitNs = 200ull * 1000 * 1000;  // bound on any mbarrier wait
+constexpr int kInjectWithholdFfn = ASF_INJECT_WITHHOLD_FFN_COPIES;
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -1011,7 +1013,7 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
                  const uint32_t *__restrict__ mask, int n_words, int32_t *__restrict__ idx_out,
                  int32_t *__restrict__ count_out, int NS, int hot_rows,
                  long long rs, int packed, float *__restrict__ part, float *__restrict__ y,
-                 Header *__restrict__ hdr, L2Next nx) {
+                 Header *__restrict__ hdr, L2Next nx, int inject) {
   constexpr int V = Vec<T>::N;
   constexpr int M = REGLU ? 3 : 2;
   constexpr int NW = kFusedWarps;
@@ -1126,13 +1128,17 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     named_sync(2, (NW + 1) * kWarp);
   }
   const int nl = s_nl;
+  int issued = 0;     // ring slots the producer has filled (its lane 0)
 
   if (warp == NW) {
     // ------------------------------------------------------------ producer --
-    // lane 0 issues one neuron's copies per ring slot
+    // lane 0 issues one neuron's copies per ring slot.  The test hook
+    // kInjectWithholdFfn makes CTA 0 issue none, so its consumers' first
+    // bounded wait runs out.
     const uint32_t row_bytes = (uint32_t)((size_t)d * sizeof(T));
     const uint64_t pol = l2_evict_first();
-    for (int i = 0; i < nl && lane == 0; ++i) {
+    const bool withhold = inject == kInjectWithholdFfn && cta == 0;
+    for (int i = 0; i < nl && lane == 0 && !withhold; ++i) {
       const int k = slist[i];
       {
         const int s = i % NS;
@@ -1140,6 +1146,8 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
           flag_error(err, kErrTimeout);
           s_fail = 1;
           break;
+        } else if (*reinterpret_cast<volatile int *>(&s_fail)) {
+          break;     // a consumer gave up: issue nothing more into the ring
         } else if ((unsigned)k >= (unsigned)n) {
           flag_error(err, kErrIndex);
           kslot[s] = -1;
@@ -1159,6 +1167,7 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
             bulk_g2s_stream(dst + d, WdT + (size_t)k * rs, row_bytes, &full[s], pol);
           }
         }
+        issued = i + 1;
       }
     }
     __syncwarp();
@@ -1192,6 +1201,7 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
         if (ok && !mbar_wait(&full[s], (uint32_t)(i / NS) & 1u, kWaitNs)) {
           if (lane == 0) flag_error(err, kErrTimeout);
           ok = false;
+          s_fail = 1;
         }
         float pg[NB], pu[NB];
 #pragma unroll
@@ -1289,6 +1299,12 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
       }
     }
   }
+  // After a wait gave up, copies the consumers no longer wait for may still be
+  // in flight: let each slot's last one land (bounded) before shared memory is
+  // released.
+  __syncthreads();
+  if (s_fail && warp == NW && lane == 0)
+    for (int i = max(0, issued - NS); i < issued; ++i) mbar_wait(&full[i % NS], (uint32_t)(i / NS) & 1u, kWaitNs);
 }
 
 // y[b][col] = sum over the G per-CTA partials, in a fixed order: lanes own 32
@@ -1417,29 +1433,8 @@ int sm_count() {
   return g_dev[dev].sms;
 }
 
-int env_flag(const char *name, int dflt) {
-  const char *v = std::getenv(name);
-  if (!v || !*v) return dflt;
-  return std::atoi(v);
-}
-
-bool pdl_enabled() {
-  static int on = env_flag("ASFFN_PDL", 1);
-  return on != 0;
-}
-size_t fused_smem_budget() {
-  static size_t kb = (size_t)env_flag("ASFFN_FUSED_SMEM_KB", (int)(kFusedSmemDefault / 1024));
-  return std::min<size_t>(std::max<size_t>(kb, 32), 220) * 1024;
-}
-bool fused_enabled() {
-  static int on = env_flag("ASFFN_FUSED", 1);
-  return on != 0;
-}
-int prefetch_enabled() {
-  static int on = env_flag("ASFFN_PREFETCH", 1);
-  return on;
-}
-
+// Process-wide test hook (asf_set_fault_injection): 0 = off.
+std::atomic<int> g_inject{0};
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                    Args... args) {
@@ -1456,7 +1451,7 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
@@ -1577,17 +1572,14 @@ cudaError_t run_pred_l2(const asf_predictor *p, int B, float thr, const float *h
   const int grid = (p->n + rpc - 1) / rpc;
   const size_t smem = (size_t)NB * p->r * 4 + ((size_t)rpc / 32 + 2) * 4;
   return launch(k_pred_l2<T, NB, (NB <= 2 ? 4 : 2), (NB <= 2 ? 4 : 2)>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W2, p->b2, h, p->r,
-                p->n, B, thr, rpc, mask, n_words_of(p->n), idx, count, hdr, prefetch_enabled());
+                p->n, B, thr, rpc, mask, n_words_of(p->n), idx, count, hdr, 1);
 }
 
 constexpr size_t kRingChunk = 32 * 1024;    // bytes per bulk copy of a ring slot
 // Shared memory of the layer-2 ring: with the register-streaming layer-1
 // kernel (one token group of x) it fits beside the previous layer's sparse
 // FFN tail, and it holds most of a CTA's W2 slice.
-size_t ring2_budget() {
-  static size_t kb = (size_t)env_flag("ASFFN_RING2_KB", 136);
-  return std::min<size_t>(std::max<size_t>(kb, 40), 200) * 1024;
-}
+constexpr size_t kRing2Budget = 136 * 1024;
 
 // rows per chunk and slots for a ring over rows of row_bytes within budget
 bool ring_shape(size_t row_bytes, size_t vec_bytes, size_t budget, int rpc, int &CR, int &NSL) {
@@ -1607,18 +1599,13 @@ cudaError_t run_pred2_ring(const asf_predictor *p, int B, float thr, const float
   const int grid = (p->n + rpc - 1) / rpc;
   const size_t vec = pred2_vec_bytes(NB, p->r, rpc);
   int CR, NSL;
-  used = ring_shape((size_t)p->r * sizeof(T), vec, ring2_budget(), rpc, CR, NSL);
+  used = ring_shape((size_t)p->r * sizeof(T), vec, kRing2Budget, rpc, CR, NSL);
   if (!used) return cudaSuccess;
   const size_t smem = ring_layout(NSL, CR, p->r, (int)sizeof(T), vec).total;
   (void)idx;
   (void)count;
   return launch(k_pred2_ring<T, NB>, dim3(grid), dim3((kRingWarps + 1) * kWarp), smem, st, (const T *)p->W2,
                 p->b2, h, p->r, p->n, B, thr, rpc, CR, NSL, mask, hdr);
-}
-
-bool ring_enabled() {
-  static int on = env_flag("ASFFN_RING", 1);
-  return on != 0;
 }
 
 // largest token group in {1, 2, 4, 8} covering B (B <= 8)
@@ -1656,6 +1643,18 @@ cudaError_t pred2_reg_any(const asf_predictor *p, int B, float thr, const float 
   }
 }
 
+// Whether layer 2 of B tokens runs the bulk-copy ring kernel, which leaves the
+// union mask for a compaction step (batches of up to 8 tokens whose W2 slice
+// fits the ring); otherwise the register-streaming kernel compacts itself.
+template <typename T>
+bool pred_leaves_mask(const asf_predictor *p, int B) {
+  if (B > 8 || n_words_of(p->n) > kCompactThreads * kCompactWords) return false;
+  const int sms = sm_count();
+  const int rpc = (p->n + sms - 1) / sms;
+  int CR, NSL;
+  return ring_shape((size_t)p->r * sizeof(T), pred2_vec_bytes(nb_cover(B), p->r, rpc), kRing2Budget, rpc, CR, NSL);
+}
+
 // Layer 1 (register-streaming kernel, token groups of up to 8), then layer 2:
 // batches of up to 8 tokens use the bulk-copy ring kernel followed by the
 // compaction kernel when the slice fits; larger batches use the
@@ -1663,12 +1662,15 @@ cudaError_t pred2_reg_any(const asf_predictor *p, int B, float thr, const float 
 template <typename T>
 cudaError_t predict_layers(const asf_predictor *p, const void *x, int B, float thr, int32_t *idx, int32_t *count,
                            Header *hdr, uint32_t *mask, float *h, cudaStream_t st, bool &mask_only) {
-  const bool ring = B <= 8 && ring_enabled() && n_words_of(p->n) <= kCompactThreads * kCompactWords;
-  mask_only = false;
+  mask_only = pred_leaves_mask<T>(p, B);
   cudaError_t e = pred1_reg_any<T>(p, x, B, h, mask, st);
   if (e != cudaSuccess) return e;
-  if (ring) e = pred2_ring_any<T>(p, B, thr, h, mask, idx, count, hdr, st, mask_only);
-  if (e != cudaSuccess || mask_only) return e;   // mask_only: the ring kernel left the union mask
+  if (mask_only) {
+    bool used = false;
+    e = pred2_ring_any<T>(p, B, thr, h, mask, idx, count, hdr, st, used);
+    if (e == cudaSuccess && !used) e = cudaErrorInvalidConfiguration;   // pred_leaves_mask said it fits
+    return e;
+  }
   return pred2_reg_any<T>(p, B, thr, h, mask, idx, count, hdr, st);
 }
 
@@ -1711,7 +1713,7 @@ cudaError_t run_down(const asf_ffn *f, int B, const int32_t *idx, const int32_t 
   const int S = down_splits(f);
   const size_t smem = (size_t)kWarps * NB * TW * 4;
   return launch(k_ffn_down<T, NB, 4>, dim3(ct, S), dim3(kThreads), smem, st, (const T *)f->WdT, a, idx, count,
-                f->d, ffn_rs(f), f->n, B, S, part, y, hdr, prefetch_enabled(), l2_next_of(f));
+                f->d, ffn_rs(f), f->n, B, S, part, y, hdr, 1, l2_next_of(f));
 }
 
 // ------------------------------------------------------------- fused ffn --
@@ -1732,7 +1734,7 @@ int fused_nl_max(const asf_ffn *f) { return (f->n + fused_grid() - 1) / fused_gr
 int fused_slots(const asf_ffn *f, int NB, int mask_words) {
   const int M = f->act == ASF_ACT_REGLU ? 3 : 2;
   for (int ns = 16; ns >= 2; --ns)
-    if (fused_layout(ns, f->d, M, esize(f->wdtype), NB, fused_nl_max(f), mask_words).total <= fused_smem_budget())
+    if (fused_layout(ns, f->d, M, esize(f->wdtype), NB, fused_nl_max(f), mask_words).total <= kFusedSmemDefault)
       return ns;
   return 0;
 }
@@ -1770,7 +1772,7 @@ cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *i
                            (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count, ml.mask,
                            ml.n_words, ml.idx_out, ml.count_out, NS,
                            (idx || ml.mask) ? std::max(0, f->hot_rows) : 0, ffn_rs(f), ffn_packed(f) ? 1 : 0, part,
-                           y, hdr, l2_next_of(f));
+                           y, hdr, l2_next_of(f), g_inject.load(std::memory_order_relaxed));
     if (e != cudaSuccess) return e;
     return launch(k_reduce_partials, dim3((f->d + kWarp - 1) / kWarp, B), dim3(kReduceWarps * kWarp), 0, st,
                   (const float *)part, G, B, f->d, y);
@@ -1808,7 +1810,7 @@ cudaError_t run_fused(const asf_ffn *f, const void *x, int B, const int32_t *idx
 // The fused kernel can rank the predictor's mask itself: the mask's words
 // still leave at least two ring slots.
 bool fused_mask_ok(const asf_ffn *f, int B) {
-  if (!fused_ok(f, B) || !fused_enabled()) return false;
+  if (!fused_ok(f, B)) return false;
   if (n_words_of(f->n) > kRankWords * kFusedWarps * kWarp) return false;   // words per ranking thread
   return fused_slots(f, fused_nb(B), n_words_of(f->n)) >= 2;
 }
@@ -1820,7 +1822,7 @@ asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, con
                  Header *hdr, unsigned char *scratch, cudaStream_t st, const MaskList &ml = MaskList()) {
   float *a = reinterpret_cast<float *>(scratch);
   float *part = reinterpret_cast<float *>(scratch + r256((size_t)f->n * B * 4));
-  if (fused_ok(f, B) && fused_enabled()) {
+  if (fused_ok(f, B)) {
     float *cpart = reinterpret_cast<float *>(scratch);
     return cuda_status(run_fused<T>(f, x, B, idx, count, cpart, y, hdr, st, ml));
   }
@@ -1848,17 +1850,22 @@ asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, con
 // scratch (mask, h) | FFN scratch.  When layer 2 leaves the union mask and the
 // fused FFN can rank it, no compaction kernel runs: the FFN kernel builds its
 // own part of the list from the mask and writes idx/count on the way.
+// parts: kPartPredict enqueues the predictor's kernels, kPartFfn the rest
+// (compaction if needed, the FFN); both together are the whole layer.
+constexpr int kPartPredict = 1, kPartFfn = 2;
 template <typename T>
 asf_status predict_ffn_t(const asf_predictor *p, const asf_ffn *f, const void *x, int B, float thr, int32_t *idx,
-                         int32_t *count, float *y, void *ws, cudaStream_t st) {
+                         int32_t *count, float *y, void *ws, cudaStream_t st, int parts) {
   unsigned char *base = static_cast<unsigned char *>(ws);
   Header *hdr = reinterpret_cast<Header *>(base);
   uint32_t *mask = reinterpret_cast<uint32_t *>(base + kHeaderBytes);
   float *h = reinterpret_cast<float *>(base + kHeaderBytes + mask_region(p));
   unsigned char *fs = base + kHeaderBytes + pred_scratch(p, B);
-  bool mask_only = false;
-  cudaError_t e = predict_layers<T>(p, x, B, thr, idx, count, hdr, mask, h, st, mask_only);
-  if (e != cudaSuccess) return ASF_ERR_CUDA;
+  bool mask_only = pred_leaves_mask<T>(p, B);
+  if (parts & kPartPredict) {
+    if (predict_layers<T>(p, x, B, thr, idx, count, hdr, mask, h, st, mask_only) != cudaSuccess) return ASF_ERR_CUDA;
+  }
+  if (!(parts & kPartFfn)) return ASF_OK;
   if (mask_only && fused_mask_ok(f, B)) {
     MaskList ml;
     ml.mask = mask;
@@ -1922,7 +1929,7 @@ asf_status noalloc_scratch(void **out) {
 // ======================================================================== //
 extern "C" {
 
-int32_t asf_version(void) { return 104; }
+int32_t asf_version(void) { return 106; }
 
 const char *asf_status_string(asf_status s) {
   switch (s) {
@@ -1987,9 +1994,12 @@ asf_status asf_sparse_ffn(const asf_ffn *ffn, const void *x, int32_t B, const in
   return ffn_t<float>(ffn, x, B, idx, count, y, hdr, scratch, (cudaStream_t)stream);
 }
 
-asf_status asf_predict_sparse_ffn(const asf_predictor *pred, const asf_ffn *ffn, const void *x, int32_t B,
-                                  float tau, int32_t *idx, int32_t *count, float *y, void *ws, size_t ws_bytes,
-                                  asf_stream_t stream) {
+}  // extern "C"
+
+namespace {
+asf_status predict_sparse_ffn_parts(const asf_predictor *pred, const asf_ffn *ffn, const void *x, int32_t B,
+                                    float tau, int32_t *idx, int32_t *count, float *y, void *ws, size_t ws_bytes,
+                                    asf_stream_t stream, int parts) {
   asf_status s = check_pred(pred);
   if (s != ASF_OK) return s;
   s = check_ffn(ffn);
@@ -2003,8 +2013,36 @@ asf_status asf_predict_sparse_ffn(const asf_predictor *pred, const asf_ffn *ffn,
   if (s != ASF_OK) return s;
   const float thr = (float)std::log((double)tau / (1.0 - (double)tau));
   if (pred->wdtype == ASF_F16)
-    return predict_ffn_t<__half>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream);
-  return predict_ffn_t<float>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream);
+    return predict_ffn_t<__half>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream, parts);
+  return predict_ffn_t<float>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream, parts);
+}
+}  // namespace
+
+extern "C" {
+
+asf_status asf_predict_sparse_ffn(const asf_predictor *pred, const asf_ffn *ffn, const void *x, int32_t B,
+                                  float tau, int32_t *idx, int32_t *count, float *y, void *ws, size_t ws_bytes,
+                                  asf_stream_t stream) {
+  return predict_sparse_ffn_parts(pred, ffn, x, B, tau, idx, count, y, ws, ws_bytes, stream,
+                                  kPartPredict | kPartFfn);
+}
+
+asf_status asf_predict_sparse_ffn_begin(const asf_predictor *pred, const asf_ffn *ffn, const void *x, int32_t B,
+                                        float tau, int32_t *idx, int32_t *count, float *y, void *ws,
+                                        size_t ws_bytes, asf_stream_t stream) {
+  return predict_sparse_ffn_parts(pred, ffn, x, B, tau, idx, count, y, ws, ws_bytes, stream, kPartPredict);
+}
+
+asf_status asf_predict_sparse_ffn_end(const asf_predictor *pred, const asf_ffn *ffn, const void *x, int32_t B,
+                                      float tau, int32_t *idx, int32_t *count, float *y, void *ws, size_t ws_bytes,
+                                      asf_stream_t stream) {
+  return predict_sparse_ffn_parts(pred, ffn, x, B, tau, idx, count, y, ws, ws_bytes, stream, kPartFfn);
+}
+
+asf_status asf_set_fault_injection(int32_t mode) {
+  if (mode != ASF_INJECT_NONE && mode != ASF_INJECT_WITHHOLD_FFN_COPIES) return ASF_ERR_INVALID_ARG;
+  g_inject.store(mode, std::memory_order_relaxed);
+  return ASF_OK;
 }
 
 asf_status asf_dense_ffn(const asf_ffn *ffn, const void *x, int32_t B, float *y, void *ws, size_t ws_bytes,

@@ -92,12 +92,25 @@ def combine_partials(y: torch.Tensor, group=None) -> torch.Tensor:
     return y
 
 
+def _torch_stream(stream):
+    """A torch stream object for a stream argument (None, torch stream or raw handle)."""
+    if stream is None or isinstance(stream, torch.cuda.Stream):
+        return stream
+    return torch.cuda.ExternalStream(int(stream))
+
+
 def sharded_layer(shard: NeuronShard, x: torch.Tensor, tau: float, idx: torch.Tensor, count: torch.Tensor,
                   y: torch.Tensor, ws: Workspace, group=None, stream=None) -> torch.Tensor:
     """One layer on this rank: predict and gather its own neurons (idx/count
-    in local ids), then combine y over the ranks."""
-    asf_predict_sparse_ffn(shard.pred, shard.ffn, x, tau, idx, count, y, ws, stream)
-    return combine_partials(y, group)
+    in local ids), then combine y over the ranks.  With a stream, the layer's
+    kernels and the all-reduce are both enqueued on it (a collective orders
+    against torch's current stream, so it is made current for the call)."""
+    ts = _torch_stream(stream)
+    asf_predict_sparse_ffn(shard.pred, shard.ffn, x, tau, idx, count, y, ws, ts)
+    if ts is None:
+        return combine_partials(y, group)
+    with torch.cuda.stream(ts):
+        return combine_partials(y, group)
 
 
 def merge_lists(per_rank: list) -> np.ndarray:

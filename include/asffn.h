@@ -165,6 +165,21 @@ ASF_API asf_status asf_predict_sparse_ffn(const asf_predictor *pred, const asf_f
                                           int32_t B, float tau, int32_t *idx, int32_t *count, float *y,
                                           void *ws, size_t ws_bytes, asf_stream_t stream);
 
+/* The same layer in two halves, for callers that put other work or timing
+ * events between the predictor and the sparse FFN.  Called in this order on
+ * one stream with identical arguments, _begin then _end enqueue exactly the
+ * kernels of asf_predict_sparse_ffn and give the same idx, count and y bit for
+ * bit.  _begin runs the predictor and leaves its result (the union mask, or
+ * for B > 8 the list itself) in the workspace; _end compacts the mask when
+ * needed and runs the sparse FFN.  Nothing else may use the workspace between
+ * the two.  Arguments, validation and errors as for asf_predict_sparse_ffn. */
+ASF_API asf_status asf_predict_sparse_ffn_begin(const asf_predictor *pred, const asf_ffn *ffn, const void *x,
+                                                int32_t B, float tau, int32_t *idx, int32_t *count, float *y,
+                                                void *ws, size_t ws_bytes, asf_stream_t stream);
+ASF_API asf_status asf_predict_sparse_ffn_end(const asf_predictor *pred, const asf_ffn *ffn, const void *x,
+                                              int32_t B, float tau, int32_t *idx, int32_t *count, float *y,
+                                              void *ws, size_t ws_bytes, asf_stream_t stream);
+
 /* Dense FFN over all n neurons (the unsparsified reference, same kernels with an
  * implicit identity index list).  Arguments as asf_sparse_ffn. */
 ASF_API asf_status asf_dense_ffn(const asf_ffn *ffn, const void *x, int32_t B, float *y, void *ws,
@@ -203,25 +218,52 @@ ASF_API asf_status asf_permute_rows(const void *src, void *dst, int32_t n_rows, 
  * a plugin inside a host framework that owns every device allocation through
  * its own pool, or a latency-critical path that cannot afford the implicit
  * device synchronisation of cudaMalloc.  This call computes exactly what
- * asf_sparse_ffn computes (same kernels), but takes its scratch from a
- * file-scope device array of ASF_NOALLOC_SCRATCH_BYTES inside the library,
- * which every GPU that loads the library holds until the process exits.
+ * asf_sparse_ffn computes (same kernels, same summation order, so the same y
+ * bit for bit), but takes its scratch from a file-scope device array of
+ * ASF_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.
  *
  *   ffn, x, B, idx, count, y   as for asf_sparse_ffn
  *   fault   optional device int32: if not NULL, it receives the raw fault bits
  *           of this call (0 = none; bit 0 = index out of range, bit 1 = timeout)
  *
+ * Size limit.  The call needs 4096 bytes of counters plus the scratch of
+ * asf_sparse_ffn: for B <= 4, G * B * d * 4 bytes of per-CTA partial sums with
+ * G = min(SM count, 256) (148 on B200); for larger B, n * B * 4 bytes of
+ * activations plus the down projection's S * B * d * 4 bytes of split sums
+ * (S <= 64 splits of the index list).  Shapes that need more than
+ * ASF_NOALLOC_SCRATCH_BYTES return ASF_ERR_UNSUPPORTED without enqueuing
+ * anything.  On B200 the 32 MiB array covers every layer with d <= 12288 and
+ * n <= 49152 at every batch up to ASF_MAX_BATCH; the largest need among them,
+ * d = 12288 at B = 4, is 29.1 MB.
+ *
  * The first call on each device looks up the array's device address for the
- * current device (cudaGetSymbolAddress); make that first call before any stream
- * capture.  Each call clears the array's counters and fault word on `stream`
- * before its kernels run.  All calls share the one array: calls that can
- * overlap on the GPU (other streams, other threads) race and must be
- * serialised by the caller.  Shapes whose scratch would exceed the array
- * (larger d, n or B) return ASF_ERR_UNSUPPORTED without enqueuing anything.
+ * current device (cudaGetSymbolAddress) and keeps it for the life of the
+ * process; make that first call before any stream capture.  The kept address
+ * is not valid across cudaDeviceReset (the library's module is reloaded in the
+ * new context): do not use this call after resetting a device.  Each call
+ * clears the array's counters and fault word on `stream` before its kernels
+ * run.  All calls share the one array: calls that can overlap on the GPU
+ * (other streams, other threads) race and must be serialised by the caller.
  * No device memory is allocated or freed, directly or by a library routine. */
-#define ASF_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define ASF_NOALLOC_SCRATCH_BYTES (32u << 20)
 ASF_API asf_status asf_sparse_ffn_noalloc(const asf_ffn *ffn, const void *x, int32_t B, const int32_t *idx,
                                           const int32_t *count, float *y, int32_t *fault, asf_stream_t stream);
+
+/* Test hook for the failure path of the bounded device waits (no counterpart
+ * in the pages).  Process-wide; read when a call enqueues its kernels.
+ *   ASF_INJECT_NONE                 normal operation (the default)
+ *   ASF_INJECT_WITHHOLD_FFN_COPIES  in the one-kernel sparse FFN (B <= 4),
+ *       CTA 0's producer issues none of its row copies, so that CTA's bounded
+ *       wait for its first row runs out (after 200 ms): the kernel records
+ *       ASF_ERR_TIMEOUT in the workspace error word, skips that CTA's rows and
+ *       returns.  y is then incomplete.  No memory is touched out of bounds,
+ *       nothing hangs and the CUDA context stays usable; the next call on the
+ *       same workspace (after asf_read_error) runs normally.
+ * Returns ASF_ERR_INVALID_ARG for any other mode. */
+#define ASF_INJECT_NONE 0
+#define ASF_INJECT_WITHHOLD_FFN_COPIES 1
+ASF_API asf_status asf_set_fault_injection(int32_t mode);
 
 /* Wait for the stream, then return (in *host_out) and clear the device error
  * word: 0, or the asf_status of the first device-side fault recorded. */
@@ -231,7 +273,8 @@ ASF_API asf_status asf_read_error(void *ws, int32_t *host_out, asf_stream_t stre
 ASF_API const char *asf_status_string(asf_status s);
 
 /* ABI version: major * 100 + minor (1.02: asf_ffn.hot_rows, asf_ffn.row_stride, asf_gather_rows;
- * 1.03: asf_ffn.l2_next; 1.04: asf_predict_sparse_ffn). */
+ * 1.03: asf_ffn.l2_next; 1.04: asf_predict_sparse_ffn; 1.05: asf_sparse_ffn_noalloc;
+ * 1.06: asf_predict_sparse_ffn_begin / _end, asf_set_fault_injection). */
 ASF_API int32_t asf_version(void);
 
 #ifdef __cplusplus

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.asf_version() == 104
+    assert lib.asf_version() == 106
     for code in range(8):
         assert lib.asf_status_string(code).decode() not in ("", "unknown status")
     assert lib.asf_status_string(99).decode() == "unknown status"
@@ -161,12 +161,37 @@ def test_sparse_ffn_rejects_bad_arguments(lib):
     assert lib.asf_dense_ffn(ctypes.byref(f), FAKE, 0, FAKE, FAKE, need, None) == L.ASF_ERR_INVALID_ARG
 
 
-def _combined(lib, p, f, x=FAKE, B=1, tau=0.5, idx=FAKE, cnt=FAKE, y=FAKE, ws=FAKE, wsb=None):
+def _combined(lib, p, f, x=FAKE, B=1, tau=0.5, idx=FAKE, cnt=FAKE, y=FAKE, ws=FAKE, wsb=None,
+              name="asf_predict_sparse_ffn"):
     if wsb is None:
         wsb = lib.asf_workspace_bytes(ctypes.byref(p), ctypes.byref(f), max(1, min(B, L.ASF_MAX_BATCH)))
-    return lib.asf_predict_sparse_ffn(ctypes.byref(p) if p is not None else None,
-                                      ctypes.byref(f) if f is not None else None, x, B, tau, idx, cnt, y,
-                                      ws, wsb, None)
+    return getattr(lib, name)(ctypes.byref(p) if p is not None else None,
+                              ctypes.byref(f) if f is not None else None, x, B, tau, idx, cnt, y,
+                              ws, wsb, None)
+
+
+@pytest.mark.parametrize("name", ["asf_predict_sparse_ffn", "asf_predict_sparse_ffn_begin",
+                                  "asf_predict_sparse_ffn_end"])
+def test_layer_calls_reject_bad_arguments(lib, name):
+    """The combined call and its two halves validate the same way."""
+    import functools
+    _combined_ = functools.partial(_combined, name=name)
+    p, f = _pred(), _ffn()
+    assert _combined_(lib, None, f, wsb=1 << 30) == L.ASF_ERR_INVALID_ARG
+    assert _combined_(lib, p, f, x=0) == L.ASF_ERR_INVALID_ARG
+    assert _combined_(lib, p, f, tau=0.0) == L.ASF_ERR_INVALID_ARG
+    assert _combined_(lib, p, f, B=33, wsb=1 << 30) == L.ASF_ERR_INVALID_ARG
+    assert _combined_(lib, _pred(n=100), _ffn(n=101), wsb=1 << 30) == L.ASF_ERR_INVALID_ARG
+    assert _combined_(lib, p, f, y=FAKE + 8) == L.ASF_ERR_MISALIGNED
+    need = lib.asf_workspace_bytes(ctypes.byref(p), ctypes.byref(f), 1)
+    assert _combined_(lib, p, f, wsb=need - 1) == L.ASF_ERR_WORKSPACE
+
+
+def test_fault_injection_modes(lib):
+    assert lib.asf_set_fault_injection(L.ASF_INJECT_WITHHOLD_FFN_COPIES) == L.ASF_OK
+    assert lib.asf_set_fault_injection(L.ASF_INJECT_NONE) == L.ASF_OK
+    for bad in (-1, 2, 99):
+        assert lib.asf_set_fault_injection(bad) == L.ASF_ERR_INVALID_ARG
 
 
 def test_combined_call_rejects_bad_arguments(lib):

@@ -64,5 +64,5 @@ def test_default_command_line(bench):
     a = bench.parse_args([])
     assert a.gpus == 1 and a.batch == 1 and a.mode == "predict" and a.impl == "ours"
     assert a.warmup >= 3 and a.steps >= 1
-    assert a.config == "llama2_7b_reglu" and a.layout == "packed"
+    assert a.config == "llama70b_reglu" and a.layout == "packed"     # the largest single-GPU stack
     assert not a.hot_prefetch and not a.l2_next

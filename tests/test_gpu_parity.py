@@ -91,22 +91,29 @@ def test_combined_call_is_bitwise_the_two_calls(layer, B):
     x = layer.Xd[rows].contiguous()
     n, d = layer.cfg.n, layer.cfg.d
     outs = []
-    for combined in (False, True):
+    for mode in ("two calls", "combined", "halves"):
         idx = torch.full((n,), -7, dtype=torch.int32, device="cuda")
         cnt = torch.full((1,), -1, dtype=torch.int32, device="cuda")
         y = torch.full((B, d), float("nan"), dtype=torch.float32, device="cuda")
-        if combined:
-            A.asf_predict_sparse_ffn(layer.pred, layer.ffn, x, layer.cfg.tau, idx, cnt, y, layer.ws)
+        args = (layer.pred, layer.ffn, x, layer.cfg.tau, idx, cnt, y, layer.ws)
+        if mode == "combined":
+            A.asf_predict_sparse_ffn(*args)
+        elif mode == "halves":
+            # the combined call in its two halves, split where a caller may put an event
+            A.asf_predict_sparse_ffn_begin(*args)
+            torch.cuda.current_stream().record_event(torch.cuda.Event())
+            A.asf_predict_sparse_ffn_end(*args)
         else:
             A.asf_predict(layer.pred, x, layer.cfg.tau, idx, cnt, layer.ws)
             A.asf_sparse_ffn(layer.ffn, x, idx, cnt, y, layer.ws)
         torch.cuda.synchronize()
         outs.append((idx.cpu().numpy(), int(cnt.item()), y.cpu().numpy()))
-    (i0, c0, y0), (i1, c1, y1) = outs
-    assert c0 == c1
-    np.testing.assert_array_equal(i0, i1)          # the list, and the untouched tail
-    assert (i1[c1:] == -7).all()
-    np.testing.assert_array_equal(y0, y1)
+    (i0, c0, y0) = outs[0]
+    for (i1, c1, y1) in outs[1:]:
+        assert c0 == c1
+        np.testing.assert_array_equal(i0, i1)          # the list, and the untouched tail
+        assert (i1[c1:] == -7).all()
+        np.testing.assert_array_equal(y0, y1)
     ref_idx = layer.oracle_idx(rows)
     np.testing.assert_array_equal(i1[:c1], ref_idx)
     assert rel_err(y1, layer.oracle_y(rows, ref_idx)) <= TOL[layer.cfg.dtype]

@@ -59,3 +59,38 @@ def test_shards_recombine_to_the_layer(layer, world, B):
     A.asf_predict_sparse_ffn(layer.pred, layer.ffn, x, cfg.tau, idx1, cnt1, y1, layer.ws)
     torch.cuda.synchronize()
     assert rel_err(y_sum.cpu().numpy(), y1.cpu().numpy()) <= TOL[cfg.dtype]
+
+
+def test_sharded_layer_orders_the_combine_on_the_callers_stream(layer, monkeypatch):
+    """With a non-default stream, the layer's kernels and the combine step (the
+    all-reduce under a process group) are enqueued on that stream, so the
+    collective cannot read y before the layer has written it."""
+    cfg = layer.cfg
+    B = 2
+    x = layer.Xd[:B].contiguous()
+    sh = SH.NeuronShard(layer.w, 0, 2)
+    ws = sh.workspace(B)
+    idx = torch.zeros(sh.n_local, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    seen = []
+    real = SH.combine_partials
+
+    def spy(y, group=None):
+        seen.append(torch.cuda.current_stream())
+        return real(y, group)
+
+    monkeypatch.setattr(SH, "combine_partials", spy)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    for stream_arg in (side, side.cuda_stream):          # torch stream and raw handle
+        y = torch.full((B, cfg.d), float("nan"), dtype=torch.float32, device="cuda")
+        SH.sharded_layer(sh, x, cfg.tau, idx, cnt, y, ws, stream=stream_arg)
+        assert seen[-1].cuda_stream == side.cuda_stream
+        side.synchronize()
+        assert torch.isfinite(y).all()
+    # without a stream, the combine runs on the current stream
+    y = torch.zeros(B, cfg.d, dtype=torch.float32, device="cuda")
+    SH.sharded_layer(sh, x, cfg.tau, idx, cnt, y, ws)
+    assert seen[-1].cuda_stream == torch.cuda.current_stream().cuda_stream
+    torch.cuda.synchronize()
+    assert A.asf_read_error(ws) == 0

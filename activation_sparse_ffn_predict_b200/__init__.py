@@ -12,6 +12,6 @@ from . import _lib  # noqa: F401
 from .api import (FFN, AsfError, Predictor, Workspace, asf_activation_counts,  # noqa: F401
                   asf_dense_ffn, asf_gather_rows, asf_hot_permutation, asf_permute_rows, asf_predict,
                   asf_predict_sparse_ffn, asf_predict_sparse_ffn_begin, asf_predict_sparse_ffn_end,
-                  asf_read_error, asf_set_fault_injection, asf_sparse_ffn, asf_sparse_ffn_noalloc,
+                  asf_predict_sparse_ffn_exchange, asf_read_error, asf_reduce_exchange, asf_set_fault_injection, asf_sparse_ffn, asf_sparse_ffn_noalloc,
                   asf_status_string, asf_version, asf_workspace_bytes, asf_workspace_init, pack_layer)
 from .stack import LayerStack  # noqa: F401

@@ -38,6 +38,14 @@ class asf_ffn(ctypes.Structure):
                 ("l2_next", c_void_p * 2), ("l2_next_bytes", ctypes.c_int64 * 2)]
 
 
+ASF_MAX_PEERS = 8
+
+
+class asf_peer_group(ctypes.Structure):
+    _fields_ = [("world", c_int32), ("rank", c_int32), ("max_batch", c_int32), ("d", c_int32),
+                ("pub", c_void_p * ASF_MAX_PEERS), ("flag", c_void_p * ASF_MAX_PEERS), ("epoch", c_void_p)]
+
+
 # name -> (restype, argtypes), exactly the declarations of include/asffn.h
 PROTOTYPES = {
     "asf_workspace_bytes": (c_size_t, [POINTER(asf_predictor), POINTER(asf_ffn), c_int32]),
@@ -54,6 +62,11 @@ PROTOTYPES = {
     "asf_predict_sparse_ffn_end": (c_int, [POINTER(asf_predictor), POINTER(asf_ffn), c_void_p, c_int32,
                                            c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                            c_void_p]),
+    "asf_predict_sparse_ffn_exchange": (c_int, [POINTER(asf_predictor), POINTER(asf_ffn), c_void_p, c_int32,
+                                                c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                                POINTER(asf_peer_group), c_void_p]),
+    "asf_reduce_exchange": (c_int, [c_void_p, c_int64, c_int32, c_int32, c_int32, POINTER(asf_peer_group),
+                                    c_int32, c_void_p, c_int64, c_void_p, c_size_t, c_void_p]),
     "asf_set_fault_injection": (c_int, [c_int32]),
     "asf_dense_ffn": (c_int, [POINTER(asf_ffn), c_void_p, c_int32, c_void_p, c_void_p, c_size_t,
                               c_void_p]),

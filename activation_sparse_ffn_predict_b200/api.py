@@ -213,6 +213,46 @@ def asf_predict_sparse_ffn_end(pred: Predictor, ffn: FFN, x: torch.Tensor, tau: 
     _layer_call("asf_predict_sparse_ffn_end", pred, ffn, x, tau, idx, count, y, ws, stream)
 
 
+def asf_predict_sparse_ffn_exchange(pred: Predictor, ffn: FFN, x: torch.Tensor, tau: float, idx: torch.Tensor,
+                                    count: torch.Tensor, y: torch.Tensor, ws: Workspace, group,
+                                    stream=None) -> None:
+    """One layer of a neuron-sharded model on this rank, with y summed over the
+    ranks of ``group`` (an ``asf_peer_group`` descriptor) through peer memory
+    inside the layer's last kernel."""
+    if x.dtype != ffn.dtype or x.dim() != 2 or x.shape[1] != ffn.d:
+        raise ValueError("x must be [B, d] in the FFN's dtype")
+    if y.shape != (x.shape[0], ffn.d):
+        raise ValueError("y must be [B, d]")
+    st = L.load().asf_predict_sparse_ffn_exchange(
+        ctypes.byref(pred.desc), ctypes.byref(ffn.desc), _dev(x, "x"), int(x.shape[0]), float(tau),
+        _dev(idx, "idx", torch.int32), _dev(count, "count", torch.int32), _dev(y, "y", torch.float32),
+        ws.ptr, ws.nbytes, ctypes.byref(group), _stream(stream))
+    check(st, "asf_predict_sparse_ffn_exchange")
+
+
+def asf_reduce_exchange(part: torch.Tensor, group, y: torch.Tensor, ws: Workspace, local_ranks: int = 1,
+                        stream=None) -> None:
+    """y = sum over ranks (rank order) of each rank's sum of its partials.
+
+    part: [G, B, d] fp32 (this rank's), or [world, G, B, d] with local_ranks ==
+    world (one process holding every rank, all run in one cooperative launch);
+    y: [B, d] or [world, B, d] accordingly."""
+    if local_ranks == 1:
+        if part.dim() != 3 or y.shape != part.shape[1:]:
+            raise ValueError("part must be [G, B, d] and y [B, d]")
+        G, B, d = part.shape
+        prs, yrs = 0, 0
+    else:
+        if part.dim() != 4 or part.shape[0] != local_ranks or y.shape != (local_ranks,) + tuple(part.shape[2:]):
+            raise ValueError("part must be [world, G, B, d] and y [world, B, d]")
+        _, G, B, d = part.shape
+        prs, yrs = G * B * d, B * d
+    st = L.load().asf_reduce_exchange(_dev(part, "part", torch.float32), prs, int(G), int(B), int(d),
+                                      ctypes.byref(group), int(local_ranks), _dev(y, "y", torch.float32), yrs,
+                                      ws.ptr, ws.nbytes, _stream(stream))
+    check(st, "asf_reduce_exchange")
+
+
 def asf_set_fault_injection(mode: int) -> None:
     """Test hook for the bounded device waits (see include/asffn.h)."""
     check(L.load().asf_set_fault_injection(int(mode)), "asf_set_fault_injection")

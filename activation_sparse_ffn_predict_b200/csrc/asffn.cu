@@ -220,13 +220,15 @@ __global__ void __launch_bounds__(kThreads)
   const int row0 = blockIdx.x * rpc;
   const int row1 = min(r, row0 + rpc);
   const int nvec = d / V;
-  // One row per warp and one token group: the warp's W1 row goes into
-  // registers before the wait.  This grid becomes resident as the previous
-  // layer's sparse FFN starts, while that kernel ranks its list and HBM is
-  // idle; a row (8 KB at d = 4096) fits that window.  (Prefetching more --
-  // this layer's W2 as well -- spilled into the FFN's row stream and delayed
-  // it.)  The next kernel reads only weights before it waits on this one.
-  const bool early = U * kWarp >= nvec && row1 - row0 <= kWarps && B <= NB;
+  // One row per warp and one token group: the first U chunks per lane of the
+  // warp's W1 row (all of it at d = 4096, half at d = 8192) go into registers
+  // before the wait.  This grid becomes resident as the previous layer's
+  // sparse FFN starts, while that kernel ranks its list and HBM is idle; about
+  // 8 KB per warp fits that window, and U = 16 keeps the kernel's registers
+  // low enough to sit beside the running FFN CTA.  (Prefetching more -- this
+  // layer's W2 as well -- spilled into the FFN's row stream and delayed it.)
+  // The next kernel reads only weights before it waits on this one.
+  const bool early = row1 - row0 <= kWarps && B <= NB;
   const int erow = row0 + warp;
   uint4 wpre[U];
   float bias_pre = 0.f;
@@ -261,6 +263,10 @@ __global__ void __launch_bounds__(kThreads)
                                  acc[b]);
         }
       }
+      // the rest of the row (rows longer than U chunks per lane), streamed now
+      if (nvec > U * kWarp)
+        row_dot<T, NB, U>(W1 + (size_t)erow * d + (size_t)U * kWarp * V, xs + (size_t)U * kWarp * V, d,
+                          nvec - U * kWarp, lane, acc);
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         const float sum = warp_sum(acc[b]);
@@ -1999,6 +2005,103 @@ __global__ void __launch_bounds__(kReduceWarps * kWarp)
 }
 
 // ======================================================================== //
+// neuron-sharded layer: the final reduction exchanged over peer memory     //
+// ======================================================================== //
+
+// Pointers of every rank's publication buffer and flag words, valid on this
+// GPU (its own, and the peers' mapped over NVLink).
+struct PeerPtrs {
+  float *pub[ASF_MAX_PEERS];
+  uint32_t *flag[ASF_MAX_PEERS];
+};
+
+// y = sum over ranks r = 0..world-1, in rank order, of rank r's sum of its G
+// partials (in order).  CTA (column block, token) first sums this rank's
+// partials as k_reduce_partials does, then warp 0 publishes the 32 sums in
+// this rank's buffer (half e & 1 for call e of the block, so a slow peer still
+// reads the previous call's half undisturbed), releases the block's flag
+// = e at system scope, waits (bounded) until every peer's flag for the block
+// reaches e, and adds all ranks' sums in rank order -- each rank computes the
+// same y bit for bit.  The exchange costs (world - 1) x 128 bytes of peer
+// reads per block, and no separate collective launch.
+//
+// blockIdx.z selects one of the ranks a process holds (1 normally; all of them
+// in the one-GPU emulation, launched cooperatively so that every block is
+// resident while it waits): rank rank0 + z, partials at part + z * part_rs,
+// output at y + z * y_rs, call counters at epoch + z * nblk.
+__global__ void __launch_bounds__(kReduceWarps * kWarp)
+    k_reduce_exchange(const float *__restrict__ part, long long part_rs, int G, int B, int d, int maxB,
+                      const __grid_constant__ PeerPtrs pp, uint32_t *__restrict__ epoch, float *__restrict__ y, long long y_rs, int world,
+                      int rank0, int32_t *__restrict__ err) {
+  __shared__ float red[kReduceWarps][kWarp];
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int col = blockIdx.x * kWarp + lane;
+  const int b = blockIdx.y;
+  const int z = blockIdx.z;
+  const int rank = rank0 + z;
+  const float *pr = part + (size_t)z * part_rs;
+  const int per = (G + kReduceWarps - 1) / kReduceWarps;
+  const int q0 = warp * per;
+  float v[kReduceMaxPerWarp];
+#pragma unroll
+  for (int u = 0; u < kReduceMaxPerWarp; ++u) {
+    const int q = q0 + u;
+    v[u] = (u < per && q < G && col < d) ? ld_cg_f32(pr + ((size_t)q * B + b) * d + col) : 0.f;
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int u = 0; u < kReduceMaxPerWarp; ++u) s += v[u];
+  red[warp][lane] = s;
+  __syncthreads();
+  if (warp != 0) return;
+  float mine = 0.f;
+#pragma unroll
+  for (int w = 0; w < kReduceWarps; ++w) mine += red[w][lane];
+  const int nbx = (d + kWarp - 1) / kWarp;
+  const int blk = b * nbx + blockIdx.x;
+  uint32_t *ep = epoch + (size_t)z * nbx * maxB + blk;
+  uint32_t e = 0;
+  if (lane == 0) {
+    e = *ep + 1u;
+    *ep = e;
+  }
+  e = __shfl_sync(0xffffffffu, e, 0);
+  const size_t half = ((size_t)(e & 1u) * maxB + b) * d;
+  if (col < d) pp.pub[rank][half + col] = mine;
+  __threadfence_system();
+  __syncwarp();
+  if (lane == 0) st_release_sys(pp.flag[rank] + blk, e);
+  // every peer's sums for this call
+  bool ok = true;
+  if (lane < world && lane != rank) {
+    const uint32_t *f = pp.flag[lane] + blk;
+    if ((int)(ld_acquire_sys(f) - e) < 0) {
+      const uint64_t t0 = global_ns();
+      while ((int)(ld_acquire_sys(f) - e) < 0) {
+        if (global_ns() - t0 > kWaitNs) {
+          ok = false;
+          break;
+        }
+      }
+    }
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && lane == 0) flag_error(err, kErrTimeout);
+  float acc = 0.f;
+  for (int h = 0; h < world; ++h) {
+    if (h == rank) {
+      acc += mine;
+    } else if (ok) {
+      (void)ld_acquire_sys(pp.flag[h] + blk);      // this lane's own acquire of the peer's release
+      acc += col < d ? ld_relaxed_sys(pp.pub[h] + half + col) : 0.f;
+    }
+  }
+  if (col < d) y[(size_t)z * y_rs + (size_t)b * d + col] = acc;
+}
+
+// ======================================================================== //
 // offline: activation counts and row permutation                           //
 // ======================================================================== //
 
@@ -2241,12 +2344,6 @@ cudaError_t run_pred_l1(const asf_predictor *p, const void *x, int B, float *h, 
   const int rpc = (p->r + sms - 1) / sms;
   const int grid = (p->r + rpc - 1) / rpc;
   const size_t smem = (size_t)NB * p->d * sizeof(T);
-  // one token, rows of 513..1024 chunks (d = 8192 in fp16): 32 chunks per lane,
-  // so the whole row still goes into registers before the dependency wait
-  const int nvec = p->d / (int)Vec<T>::N;
-  if (NB == 1 && nvec > 16 * kWarp && nvec <= 32 * kWarp)
-    return launch(k_pred_l1<T, NB, 32>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W1, p->b1, (const T *)x,
-                  p->d, p->r, B, rpc, h, mask, n_words_of(p->n));
   return launch(k_pred_l1<T, NB, (NB <= 2 ? 16 : 8)>, dim3(grid), dim3(kThreads), smem, st, (const T *)p->W1, p->b1,
                 (const T *)x, p->d, p->r, B, rpc, h, mask, n_words_of(p->n));
 }
@@ -2263,10 +2360,10 @@ cudaError_t run_pred_l2(const asf_predictor *p, int B, float thr, const float *h
 }
 
 constexpr size_t kRingChunk = 32 * 1024;    // bytes per bulk copy of a ring slot
-// Shared memory of the layer-2 ring: with the register-streaming layer-1
-// kernel (one token group of x) it fits beside the previous layer's sparse
-// FFN tail, and it holds most of a CTA's W2 slice.
-constexpr size_t kRing2Budget = 136 * 1024;
+// Shared memory of the layer-2 ring: the W2 pieces issued before the
+// dependency wait fill it (all of a CTA's slice at d_ffn = 11008, 192 KB of
+// 388 at 28672); it still fits beside the layer-1 kernel it waits on.
+constexpr size_t kRing2Budget = 200 * 1024;
 
 // rows per chunk and slots for a ring over rows of row_bytes within budget
 bool ring_shape(size_t row_bytes, size_t vec_bytes, size_t budget, int rpc, int &CR, int &NSL) {
@@ -2432,6 +2529,33 @@ cudaError_t run_down(const asf_ffn *f, int B, const int32_t *idx, const int32_t 
                 f->d, ffn_rs(f), f->n, B, S, part, y, hdr, 1, l2_next_of(f));
 }
 
+// ------------------------------------------------------- final reduce --
+// The FFN's last kernel sums its partials into y; in a neuron-sharded layer
+// (grp != nullptr) it also exchanges the ranks' sums over peer memory.
+struct Exchange {
+  const asf_peer_group *grp = nullptr;
+  int32_t *err = nullptr;
+};
+
+PeerPtrs peer_ptrs(const asf_peer_group *g) {
+  PeerPtrs pp{};
+  for (int r = 0; r < g->world; ++r) {
+    pp.pub[r] = g->pub[r];
+    pp.flag[r] = g->flag[r];
+  }
+  return pp;
+}
+
+cudaError_t launch_final_reduce(const float *part, int G, int B, int d, float *y, const Exchange &ex,
+                                cudaStream_t st) {
+  if (!ex.grp)
+    return launch(k_reduce_partials, dim3((d + kWarp - 1) / kWarp, B), dim3(kReduceWarps * kWarp), 0, st, part, G, B,
+                  d, y);
+  const asf_peer_group *g = ex.grp;
+  return launch(k_reduce_exchange, dim3((d + kWarp - 1) / kWarp, B, 1), dim3(kReduceWarps * kWarp), 0, st, part,
+                0ll, G, B, d, (int)g->max_batch, peer_ptrs(g), g->epoch, y, 0ll, (int)g->world, (int)g->rank, ex.err);
+}
+
 // ------------------------------------------------------ tensor-core ffn --
 // B in 5..32 with fp16 weights: the union contractions on tcgen05.
 bool tc_ok(const asf_ffn *f, int B) { return f->wdtype == ASF_F16 && B > 4 && B <= ASF_MAX_BATCH; }
@@ -2453,7 +2577,7 @@ cudaError_t launch_down_tc(const asf_ffn *f, int B, const int32_t *idx, const in
 }
 
 cudaError_t run_tc(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *y,
-                   Header *hdr, unsigned char *scratch, cudaStream_t st) {
+                   Header *hdr, unsigned char *scratch, cudaStream_t st, const Exchange &ex) {
   __half *a2 = reinterpret_cast<__half *>(scratch);
   float *part = reinterpret_cast<float *>(scratch + tc_a2_bytes(f, B));
   const bool reglu = f->act == ASF_ACT_REGLU;
@@ -2471,8 +2595,7 @@ cudaError_t run_tc(const asf_ffn *f, const void *x, int B, const int32_t *idx, c
     default: e = launch_down_tc<64>(f, B, idx, count, a2, part, hdr, st); break;
   }
   if (e != cudaSuccess) return e;
-  return launch(k_reduce_partials, dim3((f->d + kWarp - 1) / kWarp, B), dim3(kReduceWarps * kWarp), 0, st,
-                (const float *)part, tc_splits(f), B, f->d, y);
+  return launch_final_reduce(part, tc_splits(f), B, f->d, y, ex, st);
 }
 
 // ------------------------------------------------------------- fused ffn --
@@ -2516,7 +2639,7 @@ struct MaskList {
 
 template <typename T, int NB, int MAXQ, bool REGLU>
 cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
-                        float *y, Header *hdr, cudaStream_t st, const MaskList &ml) {
+                        float *y, Header *hdr, cudaStream_t st, const MaskList &ml, const Exchange &ex) {
   if constexpr (MAXQ * Vec<T>::N * NB > 64) {
     return cudaErrorInvalidConfiguration;
   } else {
@@ -2533,36 +2656,35 @@ cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *i
                            (idx || ml.mask) ? std::max(0, f->hot_rows) : 0, ffn_rs(f), ffn_packed(f) ? 1 : 0, part,
                            y, hdr, l2_next_of(f), g_inject.load(std::memory_order_relaxed));
     if (e != cudaSuccess) return e;
-    return launch(k_reduce_partials, dim3((f->d + kWarp - 1) / kWarp, B), dim3(kReduceWarps * kWarp), 0, st,
-                  (const float *)part, G, B, f->d, y);
+    return launch_final_reduce(part, G, B, f->d, y, ex, st);
   }
 }
 
 template <typename T, int NB, int MAXQ>
 cudaError_t run_fused_a(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
-                        float *y, Header *hdr, cudaStream_t st, const MaskList &ml) {
-  if (f->act == ASF_ACT_REGLU) return run_fused_k<T, NB, MAXQ, true>(f, x, B, idx, count, part, y, hdr, st, ml);
-  return run_fused_k<T, NB, MAXQ, false>(f, x, B, idx, count, part, y, hdr, st, ml);
+                        float *y, Header *hdr, cudaStream_t st, const MaskList &ml, const Exchange &ex) {
+  if (f->act == ASF_ACT_REGLU) return run_fused_k<T, NB, MAXQ, true>(f, x, B, idx, count, part, y, hdr, st, ml, ex);
+  return run_fused_k<T, NB, MAXQ, false>(f, x, B, idx, count, part, y, hdr, st, ml, ex);
 }
 
 template <typename T, int NB>
 cudaError_t run_fused_q(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
-                        float *y, Header *hdr, cudaStream_t st, const MaskList &ml) {
+                        float *y, Header *hdr, cudaStream_t st, const MaskList &ml, const Exchange &ex) {
   switch (fused_maxq(f)) {
-    case 1: return run_fused_a<T, NB, 1>(f, x, B, idx, count, part, y, hdr, st, ml);
-    case 2: return run_fused_a<T, NB, 2>(f, x, B, idx, count, part, y, hdr, st, ml);
-    case 4: return run_fused_a<T, NB, 4>(f, x, B, idx, count, part, y, hdr, st, ml);
-    default: return run_fused_a<T, NB, 6>(f, x, B, idx, count, part, y, hdr, st, ml);
+    case 1: return run_fused_a<T, NB, 1>(f, x, B, idx, count, part, y, hdr, st, ml, ex);
+    case 2: return run_fused_a<T, NB, 2>(f, x, B, idx, count, part, y, hdr, st, ml, ex);
+    case 4: return run_fused_a<T, NB, 4>(f, x, B, idx, count, part, y, hdr, st, ml, ex);
+    default: return run_fused_a<T, NB, 6>(f, x, B, idx, count, part, y, hdr, st, ml, ex);
   }
 }
 
 template <typename T>
 cudaError_t run_fused(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *part,
-                      float *y, Header *hdr, cudaStream_t st, const MaskList &ml) {
+                      float *y, Header *hdr, cudaStream_t st, const MaskList &ml, const Exchange &ex) {
   switch (fused_nb(B)) {
-    case 1: return run_fused_q<T, 1>(f, x, B, idx, count, part, y, hdr, st, ml);
-    case 2: return run_fused_q<T, 2>(f, x, B, idx, count, part, y, hdr, st, ml);
-    default: return run_fused_q<T, 4>(f, x, B, idx, count, part, y, hdr, st, ml);
+    case 1: return run_fused_q<T, 1>(f, x, B, idx, count, part, y, hdr, st, ml, ex);
+    case 2: return run_fused_q<T, 2>(f, x, B, idx, count, part, y, hdr, st, ml, ex);
+    default: return run_fused_q<T, 4>(f, x, B, idx, count, part, y, hdr, st, ml, ex);
   }
 }
 
@@ -2578,15 +2700,16 @@ bool fused_mask_ok(const asf_ffn *f, int B) {
 // hdr: the workspace header; scratch: this call's part of the workspace.
 template <typename T>
 asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *y,
-                 Header *hdr, unsigned char *scratch, cudaStream_t st, const MaskList &ml = MaskList()) {
+                 Header *hdr, unsigned char *scratch, cudaStream_t st, const MaskList &ml = MaskList(),
+                 const Exchange &ex = Exchange()) {
   float *a = reinterpret_cast<float *>(scratch);
   float *part = reinterpret_cast<float *>(scratch + r256((size_t)f->n * B * 4));
   if (fused_ok(f, B)) {
     float *cpart = reinterpret_cast<float *>(scratch);
-    return cuda_status(run_fused<T>(f, x, B, idx, count, cpart, y, hdr, st, ml));
+    return cuda_status(run_fused<T>(f, x, B, idx, count, cpart, y, hdr, st, ml, ex));
   }
   if (ml.mask) return ASF_ERR_UNSUPPORTED;   // callers check fused_mask_ok first
-  if (tc_ok(f, B)) return cuda_status(run_tc(f, x, B, idx, count, y, hdr, scratch, st));
+  if (tc_ok(f, B)) return cuda_status(run_tc(f, x, B, idx, count, y, hdr, scratch, st, ex));
   const int nbg = pick_nb(B, (size_t)f->d * sizeof(T));
   cudaError_t e;
   switch (nbg) {
@@ -2603,6 +2726,8 @@ asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, con
     case 4: e = run_down<T, 4>(f, B, idx, count, a, part, y, hdr, st); break;
     default: e = run_down<T, 8>(f, B, idx, count, a, part, y, hdr, st); break;
   }
+  // this path writes y itself: the exchange reads it back as a single partial
+  if (e == cudaSuccess && ex.grp) e = launch_final_reduce(y, 1, B, f->d, y, ex, st);
   return cuda_status(e);
 }
 
@@ -2615,7 +2740,8 @@ asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, con
 constexpr int kPartPredict = 1, kPartFfn = 2;
 template <typename T>
 asf_status predict_ffn_t(const asf_predictor *p, const asf_ffn *f, const void *x, int B, float thr, int32_t *idx,
-                         int32_t *count, float *y, void *ws, cudaStream_t st, int parts) {
+                         int32_t *count, float *y, void *ws, cudaStream_t st, int parts,
+                         const asf_peer_group *grp = nullptr) {
   unsigned char *base = static_cast<unsigned char *>(ws);
   Header *hdr = reinterpret_cast<Header *>(base);
   uint32_t *mask = reinterpret_cast<uint32_t *>(base + kHeaderBytes);
@@ -2626,16 +2752,19 @@ asf_status predict_ffn_t(const asf_predictor *p, const asf_ffn *f, const void *x
     if (predict_layers<T>(p, x, B, thr, idx, count, hdr, mask, h, st, mask_only) != cudaSuccess) return ASF_ERR_CUDA;
   }
   if (!(parts & kPartFfn)) return ASF_OK;
+  Exchange ex;
+  ex.grp = grp;
+  ex.err = &hdr->err;
   if (mask_only && fused_mask_ok(f, B)) {
     MaskList ml;
     ml.mask = mask;
     ml.n_words = n_words_of(p->n);
     ml.idx_out = idx;
     ml.count_out = count;
-    return ffn_t<T>(f, x, B, nullptr, nullptr, y, hdr, fs, st, ml);
+    return ffn_t<T>(f, x, B, nullptr, nullptr, y, hdr, fs, st, ml, ex);
   }
   if (mask_only && launch_compact(p, mask, idx, count, st) != cudaSuccess) return ASF_ERR_CUDA;
-  return ffn_t<T>(f, x, B, idx, count, y, hdr, fs, st);
+  return ffn_t<T>(f, x, B, idx, count, y, hdr, fs, st, MaskList(), ex);
 }
 
 template <typename T>
@@ -2757,9 +2886,21 @@ asf_status asf_sparse_ffn(const asf_ffn *ffn, const void *x, int32_t B, const in
 }  // extern "C"
 
 namespace {
+asf_status check_group(const asf_peer_group *g, int d, int B) {
+  if (!g) return ASF_ERR_INVALID_ARG;
+  if (g->world < 1 || g->world > ASF_MAX_PEERS || g->rank < 0 || g->rank >= g->world) return ASF_ERR_INVALID_ARG;
+  if (g->d != d || B < 1 || B > g->max_batch || g->max_batch > ASF_MAX_BATCH) return ASF_ERR_INVALID_ARG;
+  if (!g->epoch || !al4(g->epoch)) return ASF_ERR_INVALID_ARG;
+  for (int r = 0; r < g->world; ++r) {
+    if (!g->pub[r] || !g->flag[r]) return ASF_ERR_INVALID_ARG;
+    if (!al4(g->pub[r]) || !al4(g->flag[r])) return ASF_ERR_MISALIGNED;
+  }
+  return ASF_OK;
+}
+
 asf_status predict_sparse_ffn_parts(const asf_predictor *pred, const asf_ffn *ffn, const void *x, int32_t B,
                                     float tau, int32_t *idx, int32_t *count, float *y, void *ws, size_t ws_bytes,
-                                    asf_stream_t stream, int parts) {
+                                    asf_stream_t stream, int parts, const asf_peer_group *grp = nullptr) {
   asf_status s = check_pred(pred);
   if (s != ASF_OK) return s;
   s = check_ffn(ffn);
@@ -2771,10 +2912,14 @@ asf_status predict_sparse_ffn_parts(const asf_predictor *pred, const asf_ffn *ff
   if (!al16(x) || !al16(y) || !al4(idx) || !al4(count)) return ASF_ERR_MISALIGNED;
   s = check_ws(ws, ws_bytes, kHeaderBytes + pred_scratch(pred, B) + ffn_scratch(ffn, B));
   if (s != ASF_OK) return s;
+  if (grp) {
+    s = check_group(grp, ffn->d, B);
+    if (s != ASF_OK) return s;
+  }
   const float thr = (float)std::log((double)tau / (1.0 - (double)tau));
   if (pred->wdtype == ASF_F16)
-    return predict_ffn_t<__half>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream, parts);
-  return predict_ffn_t<float>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream, parts);
+    return predict_ffn_t<__half>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream, parts, grp);
+  return predict_ffn_t<float>(pred, ffn, x, B, thr, idx, count, y, ws, (cudaStream_t)stream, parts, grp);
 }
 }  // namespace
 
@@ -2797,6 +2942,57 @@ asf_status asf_predict_sparse_ffn_end(const asf_predictor *pred, const asf_ffn *
                                       float tau, int32_t *idx, int32_t *count, float *y, void *ws, size_t ws_bytes,
                                       asf_stream_t stream) {
   return predict_sparse_ffn_parts(pred, ffn, x, B, tau, idx, count, y, ws, ws_bytes, stream, kPartFfn);
+}
+
+asf_status asf_predict_sparse_ffn_exchange(const asf_predictor *pred, const asf_ffn *ffn, const void *x, int32_t B,
+                                           float tau, int32_t *idx, int32_t *count, float *y, void *ws,
+                                           size_t ws_bytes, const asf_peer_group *grp, asf_stream_t stream) {
+  if (!grp) return ASF_ERR_INVALID_ARG;
+  return predict_sparse_ffn_parts(pred, ffn, x, B, tau, idx, count, y, ws, ws_bytes, stream,
+                                  kPartPredict | kPartFfn, grp);
+}
+
+asf_status asf_reduce_exchange(const float *part, int64_t part_rank_stride, int32_t G, int32_t B, int32_t d,
+                               const asf_peer_group *grp, int32_t local_ranks, float *y, int64_t y_rank_stride,
+                               void *ws, size_t ws_bytes, asf_stream_t stream) {
+  if (!part || !y || G < 1 || G > kMaxGrid || d <= 0) return ASF_ERR_INVALID_ARG;
+  asf_status s = check_group(grp, d, B);
+  if (s != ASF_OK) return s;
+  if (local_ranks != 1 && local_ranks != grp->world) return ASF_ERR_INVALID_ARG;
+  if (local_ranks > 1 && grp->rank != 0) return ASF_ERR_INVALID_ARG;
+  if (local_ranks > 1 && (part_rank_stride < (int64_t)G * B * d || y_rank_stride < (int64_t)B * d))
+    return ASF_ERR_INVALID_ARG;
+  if (!al4(part) || !al4(y)) return ASF_ERR_MISALIGNED;
+  s = check_ws(ws, ws_bytes, kHeaderBytes);
+  if (s != ASF_OK) return s;
+  Header *hdr = static_cast<Header *>(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  const dim3 grid((d + kWarp - 1) / kWarp, B, local_ranks);
+  if (local_ranks == 1)
+    return cuda_status(launch(k_reduce_exchange, grid, dim3(kReduceWarps * kWarp), 0, st, part, 0ll, (int)G, (int)B,
+                              (int)d, (int)grp->max_batch, peer_ptrs(grp), grp->epoch, y, 0ll, (int)grp->world,
+                              (int)grp->rank, &hdr->err));
+  // every rank in this process: one cooperative launch, so that all blocks
+  // are resident while they wait on one another
+  int dev = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_reduce_exchange, kReduceWarps * kWarp, 0) !=
+          cudaSuccess)
+    return ASF_ERR_CUDA;
+  if ((long long)grid.x * grid.y * grid.z > (long long)per_sm * sm_count()) return ASF_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kReduceWarps * kWarp);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, k_reduce_exchange, part, (long long)part_rank_stride, (int)G, (int)B,
+                                        (int)d, (int)grp->max_batch, peer_ptrs(grp), grp->epoch, y,
+                                        (long long)y_rank_stride, (int)grp->world, 0, &hdr->err));
 }
 
 asf_status asf_set_fault_injection(int32_t mode) {

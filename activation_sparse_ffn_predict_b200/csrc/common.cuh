@@ -164,6 +164,23 @@ __device__ __forceinline__ uint32_t ticket_acq_rel(uint32_t *p) {
   return old;
 }
 
+// System-scope release store / acquire load of a flag word that other GPUs
+// read or write over peer memory, and a relaxed system-scope load of data the
+// flag guards.
+__device__ __forceinline__ void st_release_sys(uint32_t *p, uint32_t v) {
+  asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_relaxed_sys(const float *p) {
+  float v;
+  asm volatile("ld.relaxed.sys.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void flag_error(int32_t *err, int bit) {
   if (err) atomicOr(err, bit);
 }

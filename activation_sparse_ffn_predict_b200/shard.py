@@ -119,3 +119,137 @@ def merge_lists(per_rank: list) -> np.ndarray:
         return np.zeros(0, dtype=np.int32)
     return np.sort(np.concatenate([np.asarray(p, dtype=np.int64) for p in per_rank])).astype(np.int32)
 
+
+
+# --------------------------------------------------------------------------- #
+# the ranks' partial outputs exchanged over peer memory (one kernel, no NCCL)  #
+# --------------------------------------------------------------------------- #
+def exchange_sizes(d: int, max_batch: int):
+    """(publication bytes, flag words) of one rank's exchange buffers."""
+    nbx = (d + 31) // 32
+    return 2 * max_batch * d * 4, nbx * max_batch
+
+
+def group_descriptor(world: int, rank: int, max_batch: int, d: int, pub, flag, epoch):
+    """The asf_peer_group of this rank: every rank's buffer pointers in rank order."""
+    from ._lib import ASF_MAX_PEERS, asf_peer_group
+    if not (1 <= world <= ASF_MAX_PEERS) or not (0 <= rank < world):
+        raise ValueError(f"need 1 <= world <= {ASF_MAX_PEERS} and 0 <= rank < world")
+    if len(pub) != world or len(flag) != world:
+        raise ValueError("one publication buffer and one flag array per rank")
+    if any(not p for p in pub) or any(not f for f in flag) or not epoch:
+        raise ValueError("null exchange buffer")
+    g = asf_peer_group()
+    g.world, g.rank, g.max_batch, g.d = world, rank, max_batch, d
+    for r in range(world):
+        g.pub[r] = int(pub[r])
+        g.flag[r] = int(flag[r])
+    g.epoch = int(epoch)
+    return g
+
+
+class CudaIpc:
+    """Device buffers from cudaMalloc (so an IPC handle names exactly the
+    buffer) and the CUDA IPC calls that share them between processes."""
+
+    def __init__(self):
+        from cuda.bindings import runtime as rt
+        self.rt = rt
+
+    def _ok(self, res, what):
+        err = res[0] if isinstance(res, tuple) else res
+        if err != self.rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"{what} failed: {err}")
+        return res[1] if isinstance(res, tuple) and len(res) > 1 else None
+
+    def malloc_zeroed(self, nbytes: int) -> int:
+        ptr = int(self._ok(self.rt.cudaMalloc(nbytes), "cudaMalloc"))
+        self._ok(self.rt.cudaMemset(ptr, 0, nbytes), "cudaMemset")
+        return ptr
+
+    def handle(self, ptr: int) -> bytes:
+        return bytes(self._ok(self.rt.cudaIpcGetMemHandle(ptr), "cudaIpcGetMemHandle").reserved)
+
+    def open(self, handle: bytes) -> int:
+        h = self.rt.cudaIpcMemHandle_t()
+        h.reserved = handle
+        return int(self._ok(self.rt.cudaIpcOpenMemHandle(h, self.rt.cudaIpcMemLazyEnablePeerAccess),
+                            "cudaIpcOpenMemHandle"))
+
+    def close(self, ptr: int) -> None:
+        self._ok(self.rt.cudaIpcCloseMemHandle(ptr), "cudaIpcCloseMemHandle")
+
+    def free(self, ptr: int) -> None:
+        self._ok(self.rt.cudaFree(ptr), "cudaFree")
+
+    def synchronize(self) -> None:
+        self._ok(self.rt.cudaDeviceSynchronize(), "cudaDeviceSynchronize")
+
+
+class PeerGroup:
+    """The exchange buffers of the ranks of a torch.distributed group, one
+    process per GPU: this rank's publication buffer, flag words and call
+    counters, and the other ranks' buffers mapped here through CUDA IPC.
+    ``desc`` is the asf_peer_group the exchanging calls take."""
+
+    def __init__(self, d: int, max_batch: int, group=None, ipc=None):
+        self.world = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.rank = dist.get_rank(group) if dist.is_initialized() else 0
+        self.ipc = ipc if ipc is not None else CudaIpc()
+        pub_bytes, nflag = exchange_sizes(d, max_batch)
+        self.own = [self.ipc.malloc_zeroed(pub_bytes), self.ipc.malloc_zeroed(4 * nflag),
+                    self.ipc.malloc_zeroed(4 * nflag)]        # publication, flags, counters
+        self.ipc.synchronize()                                  # zeroed before any peer can look
+        mine = (self.ipc.handle(self.own[0]), self.ipc.handle(self.own[1]))
+        handles = [None] * self.world
+        if self.world > 1:
+            dist.all_gather_object(handles, mine, group=group)
+        else:
+            handles[0] = mine
+        self.opened = []
+        pub, flag = [], []
+        for r in range(self.world):
+            if r == self.rank:
+                pub.append(self.own[0])
+                flag.append(self.own[1])
+            else:
+                p, f = self.ipc.open(handles[r][0]), self.ipc.open(handles[r][1])
+                self.opened += [p, f]
+                pub.append(p)
+                flag.append(f)
+        self.desc = group_descriptor(self.world, self.rank, max_batch, d, pub, flag, self.own[2])
+        if self.world > 1:
+            dist.barrier(group=group)       # every rank mapped every buffer before the first exchange
+
+    def close(self) -> None:
+        for p in self.opened:
+            self.ipc.close(p)
+        for p in self.own:
+            self.ipc.free(p)
+        self.opened, self.own = [], []
+
+
+class EmulatedGroup:
+    """Every rank of a group held by one process on one GPU (torch buffers):
+    for exercising the exchange kernel without several GPUs
+    (asf_reduce_exchange with local_ranks == world)."""
+
+    def __init__(self, world: int, d: int, max_batch: int, device=None):
+        pub_bytes, nflag = exchange_sizes(d, max_batch)
+        dev = device if device is not None else torch.device("cuda")
+        self.pub = [torch.zeros(pub_bytes // 4, dtype=torch.float32, device=dev) for _ in range(world)]
+        self.flag = [torch.zeros(nflag, dtype=torch.int32, device=dev) for _ in range(world)]
+        self.epoch = torch.zeros(world * nflag, dtype=torch.int32, device=dev)
+        self.desc = group_descriptor(world, 0, max_batch, d, [t.data_ptr() for t in self.pub],
+                                     [t.data_ptr() for t in self.flag], self.epoch.data_ptr())
+
+
+def sharded_layer_exchange(shard: NeuronShard, x: torch.Tensor, tau: float, idx: torch.Tensor,
+                           count: torch.Tensor, y: torch.Tensor, ws: Workspace, peers: PeerGroup,
+                           stream=None) -> torch.Tensor:
+    """One layer on this rank with y summed over the ranks inside the layer's
+    last kernel (peer memory; no separate collective)."""
+    from .api import asf_predict_sparse_ffn_exchange
+    asf_predict_sparse_ffn_exchange(shard.pred, shard.ffn, x, tau, idx, count, y, ws, peers.desc,
+                                    _torch_stream(stream))
+    return y

@@ -250,6 +250,59 @@ ASF_API asf_status asf_permute_rows(const void *src, void *dst, int32_t n_rows, 
 ASF_API asf_status asf_sparse_ffn_noalloc(const asf_ffn *ffn, const void *x, int32_t B, const int32_t *idx,
                                           const int32_t *count, float *y, int32_t *fault, asf_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Neuron-sharded layer across GPUs (the layer + neuron partitioning of the
+ * "PowerInfer_x64" page's multi-GPU coordination): rank r holds the predictor
+ * rows and FFN rows of its own neurons, and the ranks' partial outputs are
+ * summed.  Here the sum is part of the layer's last kernel: each rank reduces
+ * its own per-CTA partials, publishes the result in its own buffer, and reads
+ * the other ranks' published results directly over peer memory (NVLink /
+ * NVSwitch), adding all ranks in rank order -- so every rank gets the same y,
+ * bit for bit, with no separate collective launch.
+ *
+ * Every pointer below is a device pointer valid on the calling rank's GPU:
+ * its own buffers, and the other ranks' buffers mapped into this process
+ * (CUDA IPC handles opened with peer access).  The buffers are owned by the
+ * caller and reused by every call; a rank must make the same sequence of
+ * calls (same B each time) as every other rank of the group.
+ */
+#define ASF_MAX_PEERS 8
+typedef struct {
+  int32_t world;                   /* ranks in the group, 1..ASF_MAX_PEERS */
+  int32_t rank;                    /* this rank (0 when one process emulates all ranks) */
+  int32_t max_batch;               /* B the buffers were sized for, <= ASF_MAX_BATCH */
+  int32_t d;                       /* hidden size */
+  float *pub[ASF_MAX_PEERS];       /* rank r's publication buffer: 2 * max_batch * d fp32 */
+  uint32_t *flag[ASF_MAX_PEERS];   /* rank r's flag words: ceil(d/32) * max_batch uint32 */
+  uint32_t *epoch;                 /* this rank's call counters: ceil(d/32) * max_batch uint32
+                                      (times world when one process emulates all ranks);
+                                      zero them, and every flag word, once before the first call */
+} asf_peer_group;
+
+/* One layer of a neuron-sharded model on this rank: as asf_predict_sparse_ffn
+ * over this rank's predictor and FFN rows (idx and count are local storage
+ * indices), except that y receives the sum over all ranks of their partial
+ * outputs, exchanged through grp.  A peer that does not publish within 200 ms
+ * makes the call record ASF_ERR_TIMEOUT in the workspace error word; its share
+ * is then missing from y. */
+ASF_API asf_status asf_predict_sparse_ffn_exchange(const asf_predictor *pred, const asf_ffn *ffn, const void *x,
+                                                   int32_t B, float tau, int32_t *idx, int32_t *count, float *y,
+                                                   void *ws, size_t ws_bytes, const asf_peer_group *grp,
+                                                   asf_stream_t stream);
+
+/* The exchange on its own: y = sum over ranks r (in rank order) of the sum
+ * over g < G (in order) of rank r's part[g][B][d] (fp32).  With
+ * local_ranks == 1 the call is this rank's part of the exchange; with
+ * local_ranks == grp->world one process holds every rank's partials (rank r
+ * at part + r * part_rank_stride, its y at y + r * y_rank_stride, its
+ * counters at grp->epoch + r * ceil(d/32) * max_batch) and runs all ranks in
+ * one cooperative launch on its GPU (testing the exchange without several
+ * GPUs; ASF_ERR_UNSUPPORTED if the ranks' blocks cannot all be resident).
+ * 1 <= G <= 256.  ws: a workspace (at least 4096 bytes) for the error word. */
+ASF_API asf_status asf_reduce_exchange(const float *part, int64_t part_rank_stride, int32_t G, int32_t B, int32_t d,
+                                       const asf_peer_group *grp, int32_t local_ranks, float *y,
+                                       int64_t y_rank_stride, void *ws, size_t ws_bytes, asf_stream_t stream);
+
 /* Test hook for the failure path of the bounded device waits (no counterpart
  * in the pages).  Process-wide; read when a call enqueues its kernels.
  *   ASF_INJECT_NONE                 normal operation (the default)
@@ -274,7 +327,8 @@ ASF_API const char *asf_status_string(asf_status s);
 
 /* ABI version: major * 100 + minor (1.02: asf_ffn.hot_rows, asf_ffn.row_stride, asf_gather_rows;
  * 1.03: asf_ffn.l2_next; 1.04: asf_predict_sparse_ffn; 1.05: asf_sparse_ffn_noalloc;
- * 1.06: asf_predict_sparse_ffn_begin / _end, asf_set_fault_injection). */
+ * 1.06: asf_predict_sparse_ffn_begin / _end, asf_set_fault_injection, asf_peer_group,
+ * asf_predict_sparse_ffn_exchange, asf_reduce_exchange). */
 ASF_API int32_t asf_version(void);
 
 #ifdef __cplusplus

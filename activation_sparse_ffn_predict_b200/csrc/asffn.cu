@@ -180,6 +180,28 @@ __device__ __forceinline__ void prefetch_next(const L2Next &nx, int part, int pa
   }
 }
 
+// The FFN rows of a layer's hot block (the leading rows of the hot-first
+// storage order): up to three contiguous ranges (one in the packed layout,
+// gate / up / down rows otherwise), sizes multiples of 16 bytes.
+struct HotBlock {
+  const unsigned char *p[3];
+  long long bytes[3];
+};
+
+// This CTA's share (part of parts) of an L2 prefetch of the hot block, in
+// 32 KB pieces issued by the lanes of one warp.
+__device__ __forceinline__ void prefetch_hot(const HotBlock &hb, int part, int parts) {
+  constexpr long long kPiece = 32768;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    if (!hb.p[i]) continue;
+    const long long np = (hb.bytes[i] + kPiece - 1) / kPiece;
+    for (long long q = part + (long long)parts * lane; q < np; q += (long long)parts * kWarp)
+      prefetch_l2(hb.p[i] + q * kPiece, (uint32_t)min(kPiece, hb.bytes[i] - q * kPiece));
+  }
+}
+
 // Copy n16 16-byte units from global (data written by the previous kernel,
 // read through L2) into shared memory using the first `nthreads` threads.  All
 // of a thread's loads are issued before its first store, so the copy costs one
@@ -220,15 +242,14 @@ __global__ void __launch_bounds__(kThreads)
   const int row0 = blockIdx.x * rpc;
   const int row1 = min(r, row0 + rpc);
   const int nvec = d / V;
-  // One row per warp and one token group: the first U chunks per lane of the
-  // warp's W1 row (all of it at d = 4096, half at d = 8192) go into registers
-  // before the wait.  This grid becomes resident as the previous layer's
-  // sparse FFN starts, while that kernel ranks its list and HBM is idle; about
-  // 8 KB per warp fits that window, and U = 16 keeps the kernel's registers
-  // low enough to sit beside the running FFN CTA.  (Prefetching more -- this
-  // layer's W2 as well -- spilled into the FFN's row stream and delayed it.)
-  // The next kernel reads only weights before it waits on this one.
-  const bool early = row1 - row0 <= kWarps && B <= NB;
+  // One row per warp and one token group: the warp's W1 row goes into
+  // registers before the wait.  This grid becomes resident as the previous
+  // layer's sparse FFN starts, while that kernel ranks its list and HBM is
+  // idle; a row (8 KB at d = 4096) fits that window.  (Prefetching more --
+  // this layer's W2 as well, or half of a longer row -- delayed the FFN's row
+  // stream and measured slower.)  The next kernel reads only weights before
+  // it waits on this one.
+  const bool early = U * kWarp >= nvec && row1 - row0 <= kWarps && B <= NB;
   const int erow = row0 + warp;
   uint4 wpre[U];
   float bias_pre = 0.f;
@@ -263,10 +284,6 @@ __global__ void __launch_bounds__(kThreads)
                                  acc[b]);
         }
       }
-      // the rest of the row (rows longer than U chunks per lane), streamed now
-      if (nvec > U * kWarp)
-        row_dot<T, NB, U>(W1 + (size_t)erow * d + (size_t)U * kWarp * V, xs + (size_t)U * kWarp * V, d,
-                          nvec - U * kWarp, lane, acc);
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         const float sum = warp_sum(acc[b]);
@@ -497,7 +514,7 @@ template <typename T, int NB>
 __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
     k_pred2_ring(const T *__restrict__ W2, const float *__restrict__ b2, const float *__restrict__ h, int r, int n,
                  int B, float thr, int rpc, int CR, int NSL, uint32_t *__restrict__ mask_words,
-                 Header *__restrict__ hdr) {
+                 Header *__restrict__ hdr, HotBlock hot) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int V = Vec<T>::N;
   constexpr int NT = (kRingWarps + 1) * kWarp;
@@ -526,6 +543,10 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
   if (warp == kRingWarps && lane == 0) {
     for (int i = 0; i < min(nch, NSL); ++i) ring_issue(W2, r, row0, row1, CR, NSL, i, ring, full);
   }
+  // The FFN rows of the hot block (active for most tokens) go to L2 now, while
+  // the predictor's own streams leave HBM bandwidth idle; the sparse FFN that
+  // follows then gathers its active hot rows from L2.
+  if (warp == kRingWarps) prefetch_hot(hot, blockIdx.x, gridDim.x);
   // biases are weights too: fetched before the wait, read from shared memory
   // (the consumers' named barrier below orders these stores)
   if (warp < kRingWarps)
@@ -876,34 +897,29 @@ __global__ void __launch_bounds__(kThreads)
 // many tokens on the tensor cores (tcgen05)                                //
 // ======================================================================== //
 
-// For a batch of B > 4 tokens over the union list, gate/up and down are small
-// dense GEMMs over gathered rows: [count x d].[d x B] and [d x count].[count x B].
-// On CUDA cores every weight byte then carries B fp32 FMAs, and past a few
-// tokens the FP32 pipe, not HBM, bounds the FFN.  These two kernels run the
-// contractions on the 5th-generation tensor cores instead: producer warps
-// gather the listed rows into shared memory with cp.async (16 bytes per thread,
-// any row order) directly in the swizzled layouts tcgen05.mma reads, one thread
-// issues the MMAs, and the fp32 accumulators live in tensor memory.
-//
-// Precision: x and the weights are fp16 already, so the gate/up products are
-// exact and accumulate in fp32.  The down contraction needs the activations
-// a_k (fp32) as an fp16 operand; each is carried as the sum of two fp16
-// values, hi = fp16(a) and lo = fp16(a - hi), which together hold a to about
-// 2^-22 relative, so the result stays as close to fp32 as the CUDA-core path.
-
+// For a batch of B > 4 tokens over the union list, gate/up is a small dense
+// GEMM over gathered rows: [count x d] . [d x B].  On CUDA cores every weight
+// byte then carries B fp32 FMAs, and past a few tokens the FP32 pipe, not
+// HBM, bounds it (the CUDA-core kernel also re-streams the rows once per group
+// of 8 tokens).  This kernel runs it on the 5th-generation tensor cores:
+// producer warps gather the listed rows into shared memory with cp.async (16
+// bytes per thread, any row order) directly in the 128-byte-swizzled layout
+// tcgen05.mma reads, one thread issues the MMAs, and the fp32 accumulators
+// live in tensor memory.  x and the weights are fp16 already, so the products
+// are exact and accumulate in fp32, as on the CUDA cores.  The activations go
+// to the down projection (k_ffn_down) as fp32.
 constexpr int kTcRows = 128;   // neurons per gate/up MMA tile (M)
-constexpr int kTcK = 64;       // fp16 elements of d per gate/up stage: one 128-byte swizzle row
-constexpr int kTcChunk = 32;   // list positions per activation chunk and per down stage (K)
-constexpr int kTcDW = 512;     // d columns per down CTA: four M = 128 tiles
+constexpr int kTcK = 64;       // fp16 elements of d per stage: one 128-byte swizzle row
+constexpr int kTcChunk = 32;   // list positions per share unit (one epilogue warp's rows)
+constexpr int kTcN = 16;       // tokens per MMA (N); larger batches run as several launches
 
 __device__ __forceinline__ unsigned char *align1024(unsigned char *p) {
   const uint32_t a = smem_u32(p);
   return p + (((a + 1023u) & ~1023u) - a);
 }
 
-// Gate/up kernel: NT = tokens padded to the MMA's N (16 or 32).  Stage = the
-// gate and up tiles [128 rows][64] (16 KB each, 128-byte swizzle, K-major) and
-// the x tile [NT][64].
+// Stage = the gate and up tiles [128 rows][64] (16 KB each, 128-byte swizzle,
+// K-major) and the x tile [NT][64] of the NT = 16 tokens this launch handles.
 template <int NT, bool REGLU>
 struct GuTc {
   static constexpr int W = kTcRows * kTcK * 2;
@@ -916,21 +932,19 @@ struct GuTc {
   static_assert(STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
 };
 
-// The activations of the union, written as the down kernel's B operand:
-// a2[q][row][32] fp16 for chunk q of 32 list positions, rows 0..N2/2-1 the hi
-// parts of tokens 0.., rows N2/2.. the lo parts (padding tokens and positions
-// past the list are zero).
+// a[j][g0 + b] (fp32, rows of Btot) for list position j and token b < B of
+// this launch's x (tokens g0.. of the batch).
 //
 // CTA c owns whole chunks [c*nch/G, (c+1)*nch/G) of the list.  Warps 4-7 gather
 // (one row per thread per tile), warp 8 issues the MMAs (lane 0) and owns the
 // tensor memory, warps 0-3 read the accumulators of a finished tile (lane =
-// row), apply ReLU(g + b) * u (or ReLU(u + b)) and write a2; two accumulator
+// row), apply ReLU(g + b) * u (or ReLU(u + b)) and write a; two accumulator
 // buffers let the epilogue of one tile overlap the MMAs of the next.
 template <int NT, bool REGLU>
 __global__ void __launch_bounds__(9 * kWarp)
     k_gu_tc(const __half *__restrict__ Wg, const __half *__restrict__ Wu, const float *__restrict__ bias,
             const __half *__restrict__ x, int d, long long rs, int n, int B, const int32_t *__restrict__ idx,
-            const int32_t *__restrict__ count, __half *__restrict__ a2, int N2, Header *__restrict__ hdr) {
+            const int32_t *__restrict__ count, float *__restrict__ a, int Btot, int g0, Header *__restrict__ hdr) {
   using Lg = GuTc<NT, REGLU>;
   constexpr int NS = Lg::NS;
   constexpr int MATS = REGLU ? 2 : 1;
@@ -1095,6 +1109,7 @@ __global__ void __launch_bounds__(9 * kWarp)
       const bool got = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], (uint32_t)(T >> 1) & 1u, kWaitNs));
       if (!got && lane == 0) flag_error(err, kErrTimeout);
       tc_fence_after();
+      __syncwarp();          // tensor-memory loads below are warp-synchronous
       float u[NT], g[NT];
       if (got) {
         const uint32_t cu = lane_addr + (uint32_t)(buf * MATS * NT);
@@ -1113,18 +1128,13 @@ __global__ void __launch_bounds__(9 * kWarp)
       }
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
-      if (!owned) continue;
-      const int q = j / kTcChunk;
-      const int nbt = N2 / 2;
+      if (!owned || j >= cnt) continue;
 #pragma unroll
       for (int b = 0; b < NT; ++b) {
-        if (b >= nbt) break;
-        float a = 0.f;
-        if (got && k >= 0 && b < B) a = REGLU ? fmaxf(g[b] + bk, 0.f) * u[b] : fmaxf(u[b] + bk, 0.f);
-        const __half hi = __float2half_rn(a);
-        const __half lo = __float2half_rn(a - __half2float(hi));
-        a2[((size_t)q * N2 + b) * kTcChunk + lane] = hi;
-        a2[((size_t)q * N2 + nbt + b) * kTcChunk + lane] = lo;
+        if (b >= B) break;
+        float v = 0.f;
+        if (got && k >= 0) v = REGLU ? fmaxf(g[b] + bk, 0.f) * u[b] : fmaxf(u[b] + bk, 0.f);
+        a[(size_t)j * Btot + g0 + b] = v;
       }
     }
   }
@@ -1133,398 +1143,6 @@ __global__ void __launch_bounds__(9 * kWarp)
   if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tbase, Lg::COLS);
-  }
-}
-
-// Down kernel: N2 = 2 x tokens padded (16, 32 or 64).  Stage = the W_down^T
-// tile [32 neurons][512 columns] (MN-major: 8-neuron groups of four... 64-column
-// atoms, 128-byte swizzle) and the a2 tile [N2][32] (K-major, 64-byte swizzle).
-template <int N2>
-struct DnTc {
-  static constexpr int W = kTcChunk * kTcDW * 2;
-  static constexpr int A = N2 * kTcChunk * 2;
-  static constexpr int STAGE = W + A;
-  static constexpr int NS = 5;
-  static constexpr int BAR = 1024;
-  static constexpr size_t SMEM = 1024 + BAR + (size_t)NS * STAGE;
-  static constexpr uint32_t COLS = 4 * N2;
-  static_assert(STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
-};
-
-// CTA (range r, split s) of an R x S grid accumulates, over its share of the
-// list's chunks (s-th of S), D[col][n] = sum_k WdT[k][col] a2[n][k] for the
-// 512 columns of range r: four M = 128 accumulators of N2 columns in tensor
-// memory.  Then y's partial for split s is D[col][b] + D[col][N2/2 + b] (hi +
-// lo), written to part[s][b][col]; k_reduce_partials sums the S splits in order.
-// Warps 0-3 gather (thread t: neuron t/4 of the chunk, a quarter of its 1 KB
-// row segment) and then run the epilogue; warp 4 issues the MMAs.
-template <int N2>
-__global__ void __launch_bounds__(5 * kWarp)
-    k_down_tc(const __half *__restrict__ WdT, const __half *__restrict__ a2, const int32_t *__restrict__ idx,
-              const int32_t *__restrict__ count, int d, long long rs, int n, int B, int R, int S,
-              float *__restrict__ part, Header *__restrict__ hdr) {
-  using Ld = DnTc<N2>;
-  constexpr int NS = Ld::NS;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char *smem = align1024(smem_raw);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-  uint64_t *empty = full + NS;
-  uint64_t *tfull = empty + NS;
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(tfull + 1);
-  unsigned char *stages = smem + Ld::BAR;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t *err = &hdr->err;
-
-  if (threadIdx.x == 0) {
-    for (int q = 0; q < NS; ++q) {
-      mbar_init(&full[q], 4 * kWarp);
-      mbar_init(&empty[q], 1);
-    }
-    mbar_init(&tfull[0], 1);
-    fence_mbar_init();
-  }
-  if (warp == 4) {
-    tmem_alloc(tslot, Ld::COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = *tslot;
-  pdl_wait();
-  pdl_trigger();
-
-  int cnt = n;
-  if (idx) cnt = max(0, min(ld_cg_i32(count), n));
-  const int rr = blockIdx.x % R, sp = blockIdx.x / R;
-  const int dr0 = rr * kTcDW;
-  const int nch = (cnt + kTcChunk - 1) / kTcChunk;
-  const int q0 = (int)((long long)nch * sp / S), q1 = (int)((long long)nch * (sp + 1) / S);
-  const int total = q1 - q0;
-
-  if (warp < 4) {
-    // ------------------------------------------------------------ producers --
-    const int t = threadIdx.x;
-    const int kn = t >> 2, quarter = t & 3;
-    const uint64_t pol = l2_evict_first();
-    bool ok = true;
-    for (int it = 0; it < total; ++it) {
-      const int q = q0 + it, sl = it % NS;
-      if (it >= NS && !mbar_wait(&empty[sl], (uint32_t)((it / NS) - 1) & 1u, kWaitNs)) {
-        flag_error(err, kErrTimeout);
-        ok = false;
-        break;
-      }
-      unsigned char *st = stages + (size_t)sl * Ld::STAGE;
-      const int j = q * kTcChunk + kn;
-      int k = -1;
-      if (j < cnt) {
-        k = idx ? ld_cg_i32(idx + j) : j;
-        if ((unsigned)k >= (unsigned)n) k = -1;   // flagged by the gate/up kernel
-      }
-      const __half *rowp = WdT + (size_t)max(k, 0) * rs;
-      unsigned char *wt = st + (size_t)(kn >> 3) * (kTcDW / 64) * 1024 + (size_t)(kn & 7) * 128;
-#pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const int ci = quarter * 16 + cc;            // 16-byte chunk of the 1 KB segment
-        const int col = dr0 + ci * 8;
-        const bool in = k >= 0 && col < d;
-        cp_async16(wt + (size_t)(ci >> 3) * 1024 + (((ci & 7) ^ (kn & 7)) << 4),
-                   in ? (const void *)(rowp + col) : (const void *)WdT, in ? 16u : 0u, pol);
-      }
-      unsigned char *at = st + Ld::W;
-      for (int qq = t; qq < N2 * 4; qq += 4 * kWarp) {
-        const int row = qq >> 2, c = qq & 3;
-        cp_async16(at + row * 64 + ((c ^ ((row >> 1) & 3)) << 4), a2 + ((size_t)q * N2 + row) * kTcChunk + c * 8,
-                   16u);
-      }
-      cp_async_commit();
-      if (it >= NS - 1) {
-        cp_async_wait<NS - 1>();
-        fence_proxy_async_smem();
-        mbar_arrive(&full[(it - (NS - 1)) % NS]);
-      }
-    }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (ok)
-      for (int it = max(0, total - (NS - 1)); it < total; ++it) mbar_arrive(&full[it % NS]);
-    // ------------------------------------------------------------- epilogue --
-    bool got = total > 0 && ok;
-    if (got) got = __all_sync(0xffffffffu, mbar_wait(&tfull[0], 0u, kWaitNs));
-    if (total > 0 && !got && lane == 0) flag_error(err, kErrTimeout);
-    tc_fence_after();
-    const uint32_t lane_addr = tbase + ((uint32_t)(kWarp * warp) << 16);
-#pragma unroll 1
-    for (int i = 0; i < kTcDW / kTcRows; ++i) {
-      const int col = dr0 + i * kTcRows + kWarp * warp + lane;
-      float v[N2];
-      if (got) {
-#pragma unroll
-        for (int h = 0; h < N2 / 16; ++h) {
-          float w[16];
-          tmem_ld16(lane_addr + (uint32_t)(i * N2 + 16 * h), w);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[16 * h + e] = w[e];
-        }
-      }
-      if (col < d) {
-#pragma unroll
-        for (int b = 0; b < N2 / 2; ++b)
-          if (b < B) part[((size_t)sp * B + b) * d + col] = got ? v[b] + v[N2 / 2 + b] : 0.f;
-      }
-    }
-  } else {
-    // ------------------------------------------------------------------ MMA --
-    if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_f16(kTcRows, N2, 1, 0);
-      bool ok = true;
-      for (int it = 0; it < total; ++it) {
-        const int sl = it % NS;
-        if (!mbar_wait(&full[sl], (uint32_t)(it / NS) & 1u, kWaitNs)) {
-          flag_error(err, kErrTimeout);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        unsigned char *st = stages + (size_t)sl * Ld::STAGE;
-#pragma unroll
-        for (int kk = 0; kk < kTcChunk / 16; ++kk) {
-          const uint64_t bd = umma_desc(st + Ld::W + kk * 32, 16, 512, kSwz64);
-#pragma unroll
-          for (int i = 0; i < kTcDW / kTcRows; ++i) {
-            // neurons 16kk..16kk+15 = 8-row groups 2kk, 2kk+1; columns 128i.. = atoms 2i, 2i+1
-            const uint64_t ad = umma_desc(st + (size_t)((2 * kk) * (kTcDW / 64) + 2 * i) * 1024, 1024,
-                                          (kTcDW / 64) * 1024, kSwz128);
-            umma_f16(tbase + (uint32_t)(i * N2), ad, bd, idesc, (it | kk) != 0);
-          }
-        }
-        umma_commit(&empty[sl]);
-      }
-      if (ok && total > 0) umma_commit(&tfull[0]);
-    }
-    __syncwarp();
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 4) {
-    tc_fence_after();
-    tmem_dealloc(tbase, Ld::COLS);
-  }
-}
-
-// Predictor layer 2 of B > 8 tokens on the tensor cores.  h [B][r] fp32 (from
-// the layer-1 kernel) is first rewritten as the MMA's B operand: h2[q][row][64]
-// fp16 for chunk q of 64 hidden units, rows 0..N2/2-1 the hi parts of tokens
-// 0.., rows N2/2.. the lo parts (hi + lo = h to about 2^-22 relative).
-__global__ void __launch_bounds__(kThreads)
-    k_h_to_h2(const float *__restrict__ h, int B, int r, int N2, __half *__restrict__ h2) {
-  pdl_wait();
-  pdl_trigger();
-  const int nbt = N2 / 2;
-  const int per = N2 * kTcK;
-  const int total = (r + kTcK - 1) / kTcK * per;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-    const int q = i / per, rem = i - q * per;
-    const int row = rem / kTcK, e = q * kTcK + (rem - row * kTcK);
-    const int b = row < nbt ? row : row - nbt;
-    const float v = (b < B && e < r) ? __ldcg(h + (size_t)b * r + e) : 0.f;
-    const __half hi = __float2half_rn(v);
-    h2[i] = row < nbt ? hi : __float2half_rn(v - __half2float(hi));
-  }
-}
-
-template <int N2>
-struct P2Tc {
-  static constexpr int W = kTcRows * kTcK * 2;
-  static constexpr int H = N2 * kTcK * 2;
-  static constexpr int STAGE = W + H;
-  static constexpr int NS = 8;
-  static constexpr int BAR = 1024;
-  static constexpr size_t SMEM = 1024 + BAR + (size_t)NS * STAGE;
-  static constexpr uint32_t COLS = 2 * N2;                 // double-buffered
-  static_assert(STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
-};
-
-// z = W2 h + b2 and the union mask for B tokens: CTA c owns whole mask words
-// [c*nw/G, (c+1)*nw/G), i.e. rows in tiles of 128 (K = r in stages of 64).
-// Warps 4-7 stream W2 rows and the h2 chunk, warp 8 issues the MMAs, warps 0-3
-// read z (lane = row; hi + lo columns summed per token), compare with the
-// threshold and write the words they own (32 rows = one word per warp).
-template <int N2>
-__global__ void __launch_bounds__(9 * kWarp)
-    k_pred2_tc(const __half *__restrict__ W2, const float *__restrict__ b2, const __half *__restrict__ h2, int r,
-               int n, int B, float thr, uint32_t *__restrict__ mask_words, Header *__restrict__ hdr) {
-  using Lp = P2Tc<N2>;
-  constexpr int NS = Lp::NS;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char *smem = align1024(smem_raw);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-  uint64_t *empty = full + NS;
-  uint64_t *tfull = empty + NS;
-  uint64_t *tempty = tfull + 2;
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(tempty + 2);
-  unsigned char *stages = smem + Lp::BAR;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t *err = &hdr->err;
-
-  if (threadIdx.x == 0) {
-    for (int q = 0; q < NS; ++q) {
-      mbar_init(&full[q], 4 * kWarp);
-      mbar_init(&empty[q], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4 * kWarp);
-    }
-    fence_mbar_init();
-  }
-  if (warp == 8) {
-    tmem_alloc(tslot, Lp::COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = *tslot;
-
-  const int nw = (n + 31) / 32;
-  const int own0 = 32 * (int)((long long)nw * blockIdx.x / gridDim.x);
-  const int own1 = 32 * (int)((long long)nw * (blockIdx.x + 1) / gridDim.x);
-  const int ntiles = (own1 - own0 + kTcRows - 1) / kTcRows;
-  const int nK = (r + kTcK - 1) / kTcK;
-  const int total = ntiles * nK;
-
-  pdl_trigger();
-  if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ producers --
-    // W2 does not depend on the previous kernels: the first P stages' W2 tiles
-    // are issued before the dependency wait, their h2 chunks after it; then
-    // every stage is one cp.async group, released NS - 1 groups later.
-    const int t = threadIdx.x - 4 * kWarp;
-    const uint64_t pol = l2_evict_first();
-    auto issue_w2 = [&](int it) {
-      const int T = it / nK, kc = it - T * nK;
-      unsigned char *st = stages + (size_t)(it % NS) * Lp::STAGE;
-      const int row = own0 + T * kTcRows + t;
-      const bool rin = row < own1 && row < n;
-      const int col0 = kc * kTcK;
-      const __half *rowp = W2 + (size_t)(rin ? row : 0) * r + col0;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const bool in = rin && col0 + c * 8 < r;
-        cp_async16(st + (size_t)t * 128 + ((c ^ (t & 7)) << 4), in ? (const void *)(rowp + c * 8) : (const void *)W2,
-                   in ? 16u : 0u, pol);
-      }
-    };
-    auto issue_h2 = [&](int it) {
-      const int kc = it % nK;
-      unsigned char *ht = stages + (size_t)(it % NS) * Lp::STAGE + Lp::W;
-      for (int qq = t; qq < N2 * 8; qq += 4 * kWarp) {
-        const int hrow = qq >> 3, c = qq & 7;
-        cp_async16(ht + hrow * 128 + ((c ^ (hrow & 7)) << 4), h2 + ((size_t)kc * N2 + hrow) * kTcK + c * 8, 16u);
-      }
-    };
-    const int P = min(NS, total);
-    for (int it = 0; it < P; ++it) issue_w2(it);
-    pdl_wait();
-    for (int it = 0; it < P; ++it) issue_h2(it);
-    cp_async_commit();
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    for (int it = 0; it < P; ++it) mbar_arrive(&full[it]);
-    bool ok = true;
-    for (int it = P; it < total; ++it) {
-      const int sl = it % NS;
-      if (!mbar_wait(&empty[sl], (uint32_t)((it / NS) - 1) & 1u, kWaitNs)) {
-        flag_error(err, kErrTimeout);
-        ok = false;
-        break;
-      }
-      issue_w2(it);
-      issue_h2(it);
-      cp_async_commit();
-      if (it - (NS - 1) >= P) {
-        cp_async_wait<NS - 1>();
-        fence_proxy_async_smem();
-        mbar_arrive(&full[(it - (NS - 1)) % NS]);
-      }
-    }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (ok)
-      for (int it = max(P, total - (NS - 1)); it < total; ++it) mbar_arrive(&full[it % NS]);
-  } else if (warp == 8) {
-    // ------------------------------------------------------------------ MMA --
-    if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_f16(kTcRows, N2, 0, 0);
-      bool ok = true;
-      for (int T = 0; T < ntiles && ok; ++T) {
-        const int buf = T & 1;
-        if (T >= 2 && !mbar_wait(&tempty[buf], (uint32_t)((T >> 1) - 1) & 1u, kWaitNs)) {
-          flag_error(err, kErrTimeout);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t dz = tbase + (uint32_t)(buf * N2);
-        for (int kc = 0; kc < nK; ++kc) {
-          const int it = T * nK + kc, sl = it % NS;
-          if (!mbar_wait(&full[sl], (uint32_t)(it / NS) & 1u, kWaitNs)) {
-            flag_error(err, kErrTimeout);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          unsigned char *st = stages + (size_t)sl * Lp::STAGE;
-          const uint64_t dw = umma_desc(st, 16, 1024, kSwz128);
-          const uint64_t dh = umma_desc(st + Lp::W, 16, 1024, kSwz128);
-#pragma unroll
-          for (int k4 = 0; k4 < kTcK / 16; ++k4) umma_f16(dz, dw + 2 * k4, dh + 2 * k4, idesc, (kc | k4) != 0);
-          umma_commit(&empty[sl]);
-        }
-        if (ok) umma_commit(&tfull[buf]);
-      }
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------- epilogue --
-    pdl_wait();
-    const int rr = threadIdx.x;
-    const uint32_t lane_addr = tbase + ((uint32_t)(kWarp * warp) << 16);
-    for (int T = 0; T < ntiles; ++T) {
-      const int buf = T & 1;
-      const int row = own0 + T * kTcRows + rr;
-      const bool owned = row < own1;             // uniform over the warp
-      const float bias = (owned && row < n) ? __ldg(b2 + row) : 0.f;
-      const bool got = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], (uint32_t)(T >> 1) & 1u, kWaitNs));
-      if (!got && lane == 0) flag_error(err, kErrTimeout);
-      tc_fence_after();
-      float v[N2];
-      if (got) {
-#pragma unroll
-        for (int hh = 0; hh < N2 / 16; ++hh) {
-          float w[16];
-          tmem_ld16(lane_addr + (uint32_t)(buf * N2 + 16 * hh), w);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[16 * hh + e] = w[e];
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&tempty[buf]);
-      if (!owned) continue;
-      bool on = false;
-#pragma unroll
-      for (int b = 0; b < N2 / 2; ++b)
-        if (got && b < B && row < n) on |= (v[b] + v[N2 / 2 + b]) + bias > thr;
-      const uint32_t word = __ballot_sync(0xffffffffu, on);
-      if (lane == 0) mask_words[row >> 5] = word;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 8) {
-    tc_fence_after();
-    tmem_dealloc(tbase, Lp::COLS);
   }
 }
 
@@ -2248,36 +1866,12 @@ bool ffn_packed(const asf_ffn *f) {
   return static_cast<const char *>(f->WdT) == first + (size_t)(M - 1) * rb;
 }
 
-// Tensor-core path (fp16 weights): N of the MMAs that carry B tokens as hi/lo pairs.
-int tc_n2(int B) { return B <= 8 ? 16 : B <= 16 ? 32 : 64; }
-
-// Predictor layer 2 runs on the tensor cores for B > 8 tokens with fp16 weights.
-bool pred_tc(const asf_predictor *p, int B) { return p->wdtype == ASF_F16 && B > 8; }
-size_t pred_h2_bytes(const asf_predictor *p, int B) {
-  return pred_tc(p, B) ? r256((size_t)((p->r + kTcK - 1) / kTcK) * tc_n2(B) * kTcK * 2) : 0;
-}
-// mask words | h [B][r] fp32 | h2 (tensor-core operand, B > 8)
-size_t pred_scratch(const asf_predictor *p, int B) {
-  return mask_region(p) + r256((size_t)B * p->r * 4) + pred_h2_bytes(p, B);
-}
-
-// Tensor-core FFN for B > 4 (fp16 weights): a2 activations and split partials.
-int tc_ranges(const asf_ffn *f) { return (f->d + kTcDW - 1) / kTcDW; }
-int tc_splits(const asf_ffn *f) {
-  const int R = tc_ranges(f);
-  return std::max(1, std::min(kMaxGrid, sm_count() / R));
-}
-size_t tc_a2_bytes(const asf_ffn *f, int B) {
-  return r256((size_t)((f->n + kTcChunk - 1) / kTcChunk) * tc_n2(B) * kTcChunk * 2);
-}
-size_t tc_scratch(const asf_ffn *f, int B) {
-  return tc_a2_bytes(f, B) + r256((size_t)tc_splits(f) * B * f->d * 4);
-}
+size_t pred_scratch(const asf_predictor *p, int B) { return mask_region(p) + r256((size_t)B * p->r * 4); }
 
 size_t ffn_scratch(const asf_ffn *f, int B) {
   const size_t two_kernel = r256((size_t)f->n * B * 4) + r256((size_t)down_splits(f) * B * f->d * 4);
   const size_t fused = r256((size_t)std::min(sm_count(), kMaxGrid) * B * f->d * 4);
-  return std::max({two_kernel, fused, f->wdtype == ASF_F16 ? tc_scratch(f, B) : (size_t)0});
+  return std::max(two_kernel, fused);
 }
 
 asf_status check_pred(const asf_predictor *p) {
@@ -2360,10 +1954,11 @@ cudaError_t run_pred_l2(const asf_predictor *p, int B, float thr, const float *h
 }
 
 constexpr size_t kRingChunk = 32 * 1024;    // bytes per bulk copy of a ring slot
-// Shared memory of the layer-2 ring: the W2 pieces issued before the
-// dependency wait fill it (all of a CTA's slice at d_ffn = 11008, 192 KB of
-// 388 at 28672); it still fits beside the layer-1 kernel it waits on.
-constexpr size_t kRing2Budget = 200 * 1024;
+// Shared memory of the layer-2 ring: with the register-streaming layer-1
+// kernel (one token group of x) it fits beside the previous layer's sparse
+// FFN tail, and it holds most of a CTA's W2 slice.  (A 200 KB ring, holding
+// more of the slice before the wait, measured 1.5-4% slower end to end.)
+constexpr size_t kRing2Budget = 136 * 1024;
 
 // rows per chunk and slots for a ring over rows of row_bytes within budget
 bool ring_shape(size_t row_bytes, size_t vec_bytes, size_t budget, int rpc, int &CR, int &NSL) {
@@ -2377,7 +1972,7 @@ bool ring_shape(size_t row_bytes, size_t vec_bytes, size_t budget, int rpc, int 
 
 template <typename T, int NB>
 cudaError_t run_pred2_ring(const asf_predictor *p, int B, float thr, const float *h, uint32_t *mask, int32_t *idx,
-                           int32_t *count, Header *hdr, cudaStream_t st, bool &used) {
+                           int32_t *count, Header *hdr, cudaStream_t st, bool &used, const HotBlock &hot) {
   const int sms = sm_count();
   const int rpc = (p->n + sms - 1) / sms;
   const int grid = (p->n + rpc - 1) / rpc;
@@ -2389,7 +1984,7 @@ cudaError_t run_pred2_ring(const asf_predictor *p, int B, float thr, const float
   (void)idx;
   (void)count;
   return launch(k_pred2_ring<T, NB>, dim3(grid), dim3((kRingWarps + 1) * kWarp), smem, st, (const T *)p->W2,
-                p->b2, h, p->r, p->n, B, thr, rpc, CR, NSL, mask, hdr);
+                p->b2, h, p->r, p->n, B, thr, rpc, CR, NSL, mask, hdr, hot);
 }
 
 // largest token group in {1, 2, 4, 8} covering B (B <= 8)
@@ -2397,12 +1992,12 @@ inline int nb_cover(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 8; }
 
 template <typename T>
 cudaError_t pred2_ring_any(const asf_predictor *p, int B, float thr, const float *h, uint32_t *mask, int32_t *idx,
-                           int32_t *count, Header *hdr, cudaStream_t st, bool &used) {
+                           int32_t *count, Header *hdr, cudaStream_t st, bool &used, const HotBlock &hot) {
   switch (nb_cover(B)) {
-    case 1: return run_pred2_ring<T, 1>(p, B, thr, h, mask, idx, count, hdr, st, used);
-    case 2: return run_pred2_ring<T, 2>(p, B, thr, h, mask, idx, count, hdr, st, used);
-    case 4: return run_pred2_ring<T, 4>(p, B, thr, h, mask, idx, count, hdr, st, used);
-    default: return run_pred2_ring<T, 8>(p, B, thr, h, mask, idx, count, hdr, st, used);
+    case 1: return run_pred2_ring<T, 1>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
+    case 2: return run_pred2_ring<T, 2>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
+    case 4: return run_pred2_ring<T, 4>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
+    default: return run_pred2_ring<T, 8>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
   }
 }
 
@@ -2432,9 +2027,7 @@ cudaError_t pred2_reg_any(const asf_predictor *p, int B, float thr, const float 
 // fits the ring); otherwise the register-streaming kernel compacts itself.
 template <typename T>
 bool pred_leaves_mask(const asf_predictor *p, int B) {
-  if (n_words_of(p->n) > kCompactThreads * kCompactWords) return false;
-  if (pred_tc(p, B)) return true;
-  if (B > 8) return false;
+  if (B > 8 || n_words_of(p->n) > kCompactThreads * kCompactWords) return false;
   const int sms = sm_count();
   const int rpc = (p->n + sms - 1) / sms;
   int CR, NSL;
@@ -2445,42 +2038,16 @@ bool pred_leaves_mask(const asf_predictor *p, int B) {
 // batches of up to 8 tokens use the bulk-copy ring kernel followed by the
 // compaction kernel when the slice fits; larger batches use the
 // register-streaming layer-2 kernel, which compacts in its last CTA.
-template <int N2>
-cudaError_t launch_pred2_tc(const asf_predictor *p, int B, float thr, const __half *h2, uint32_t *mask, Header *hdr,
-                            cudaStream_t st) {
-  return launch(k_pred2_tc<N2>, dim3(std::min(sm_count(), kMaxGrid)), dim3(9 * kWarp), P2Tc<N2>::SMEM, st,
-                (const __half *)p->W2, p->b2, h2, p->r, p->n, B, thr, mask, hdr);
-}
-
-// Layer 2 of B > 8 tokens on the tensor cores: h -> h2 (hi/lo fp16), then the
-// MMA kernel writes every union-mask word.
-cudaError_t pred2_tc_any(const asf_predictor *p, int B, float thr, const float *h, __half *h2, uint32_t *mask,
-                         Header *hdr, cudaStream_t st) {
-  const int N2 = tc_n2(B);
-  const int total = (p->r + kTcK - 1) / kTcK * N2 * kTcK;
-  cudaError_t e = launch(k_h_to_h2, dim3(std::min(sm_count(), (total + kThreads - 1) / kThreads)), dim3(kThreads), 0,
-                         st, h, B, p->r, N2, h2);
-  if (e != cudaSuccess) return e;
-  switch (N2) {
-    case 16: return launch_pred2_tc<16>(p, B, thr, h2, mask, hdr, st);
-    case 32: return launch_pred2_tc<32>(p, B, thr, h2, mask, hdr, st);
-    default: return launch_pred2_tc<64>(p, B, thr, h2, mask, hdr, st);
-  }
-}
-
 template <typename T>
 cudaError_t predict_layers(const asf_predictor *p, const void *x, int B, float thr, int32_t *idx, int32_t *count,
-                           Header *hdr, uint32_t *mask, float *h, cudaStream_t st, bool &mask_only) {
+                           Header *hdr, uint32_t *mask, float *h, cudaStream_t st, bool &mask_only,
+                           const HotBlock &hot = HotBlock()) {
   mask_only = pred_leaves_mask<T>(p, B);
   cudaError_t e = pred1_reg_any<T>(p, x, B, h, mask, st);
   if (e != cudaSuccess) return e;
-  if (pred_tc(p, B)) {
-    __half *h2 = reinterpret_cast<__half *>(reinterpret_cast<unsigned char *>(h) + r256((size_t)B * p->r * 4));
-    return pred2_tc_any(p, B, thr, h, h2, mask, hdr, st);
-  }
   if (mask_only) {
     bool used = false;
-    e = pred2_ring_any<T>(p, B, thr, h, mask, idx, count, hdr, st, used);
+    e = pred2_ring_any<T>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
     if (e == cudaSuccess && !used) e = cudaErrorInvalidConfiguration;   // pred_leaves_mask said it fits
     return e;
   }
@@ -2557,45 +2124,35 @@ cudaError_t launch_final_reduce(const float *part, int G, int B, int d, float *y
 }
 
 // ------------------------------------------------------ tensor-core ffn --
-// B in 5..32 with fp16 weights: the union contractions on tcgen05.
+// B in 5..32 with fp16 weights: gate/up on tcgen05 in launches of 16 tokens
+// (one pass over the rows for B <= 16, two for B <= 32), then the down
+// projection over the same list on the CUDA cores.
 bool tc_ok(const asf_ffn *f, int B) { return f->wdtype == ASF_F16 && B > 4 && B <= ASF_MAX_BATCH; }
 
-template <int NT, bool REGLU>
-cudaError_t launch_gu_tc(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count,
-                         __half *a2, Header *hdr, cudaStream_t st) {
-  return launch(k_gu_tc<NT, REGLU>, dim3(std::min(sm_count(), kMaxGrid)), dim3(9 * kWarp), GuTc<NT, REGLU>::SMEM,
-                st, (const __half *)f->Wg, (const __half *)f->Wu, f->bias, (const __half *)x, f->d, ffn_rs(f), f->n,
-                B, idx, count, a2, tc_n2(B), hdr);
-}
-
-template <int N2>
-cudaError_t launch_down_tc(const asf_ffn *f, int B, const int32_t *idx, const int32_t *count, const __half *a2,
-                           float *part, Header *hdr, cudaStream_t st) {
-  const int R = tc_ranges(f), S = tc_splits(f);
-  return launch(k_down_tc<N2>, dim3(R * S), dim3(5 * kWarp), DnTc<N2>::SMEM, st, (const __half *)f->WdT, a2, idx,
-                count, f->d, ffn_rs(f), f->n, B, R, S, part, hdr);
+template <bool REGLU>
+cudaError_t launch_gu_tc(const asf_ffn *f, const __half *x, int Bh, int Btot, int g0, const int32_t *idx,
+                         const int32_t *count, float *a, Header *hdr, cudaStream_t st) {
+  return launch(k_gu_tc<kTcN, REGLU>, dim3(std::min(sm_count(), kMaxGrid)), dim3(9 * kWarp),
+                GuTc<kTcN, REGLU>::SMEM, st, (const __half *)f->Wg, (const __half *)f->Wu, f->bias, x, f->d,
+                ffn_rs(f), f->n, Bh, idx, count, a, Btot, g0, hdr);
 }
 
 cudaError_t run_tc(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *y,
                    Header *hdr, unsigned char *scratch, cudaStream_t st, const Exchange &ex) {
-  __half *a2 = reinterpret_cast<__half *>(scratch);
-  float *part = reinterpret_cast<float *>(scratch + tc_a2_bytes(f, B));
+  float *a = reinterpret_cast<float *>(scratch);
+  float *part = reinterpret_cast<float *>(scratch + r256((size_t)f->n * B * 4));
   const bool reglu = f->act == ASF_ACT_REGLU;
-  cudaError_t e;
-  if (B <= 16)
-    e = reglu ? launch_gu_tc<16, true>(f, x, B, idx, count, a2, hdr, st)
-              : launch_gu_tc<16, false>(f, x, B, idx, count, a2, hdr, st);
-  else
-    e = reglu ? launch_gu_tc<32, true>(f, x, B, idx, count, a2, hdr, st)
-              : launch_gu_tc<32, false>(f, x, B, idx, count, a2, hdr, st);
-  if (e != cudaSuccess) return e;
-  switch (tc_n2(B)) {
-    case 16: e = launch_down_tc<16>(f, B, idx, count, a2, part, hdr, st); break;
-    case 32: e = launch_down_tc<32>(f, B, idx, count, a2, part, hdr, st); break;
-    default: e = launch_down_tc<64>(f, B, idx, count, a2, part, hdr, st); break;
+  cudaError_t e = cudaSuccess;
+  for (int g0 = 0; g0 < B && e == cudaSuccess; g0 += kTcN) {
+    const int Bh = std::min(kTcN, B - g0);
+    const __half *xg = static_cast<const __half *>(x) + (size_t)g0 * f->d;
+    e = reglu ? launch_gu_tc<true>(f, xg, Bh, B, g0, idx, count, a, hdr, st)
+              : launch_gu_tc<false>(f, xg, Bh, B, g0, idx, count, a, hdr, st);
   }
   if (e != cudaSuccess) return e;
-  return launch_final_reduce(part, tc_splits(f), B, f->d, y, ex, st);
+  e = run_down<__half, 8>(f, B, idx, count, a, part, y, hdr, st);
+  if (e == cudaSuccess && ex.grp) e = launch_final_reduce(y, 1, B, f->d, y, ex, st);
+  return e;
 }
 
 // ------------------------------------------------------------- fused ffn --
@@ -2653,7 +2210,7 @@ cudaError_t run_fused_k(const asf_ffn *f, const void *x, int B, const int32_t *i
     cudaError_t e = launch(kern, dim3(G), dim3(threads), L.total, st, (const T *)f->Wg, (const T *)f->Wu,
                            (const T *)f->WdT, f->bias, (const T *)x, f->d, f->n, B, idx, count, ml.mask,
                            ml.n_words, ml.idx_out, ml.count_out, NS,
-                           (idx || ml.mask) ? std::max(0, f->hot_rows) : 0, ffn_rs(f), ffn_packed(f) ? 1 : 0, part,
+                           idx ? std::max(0, f->hot_rows) : 0, ffn_rs(f), ffn_packed(f) ? 1 : 0, part,
                            y, hdr, l2_next_of(f), g_inject.load(std::memory_order_relaxed));
     if (e != cudaSuccess) return e;
     return launch_final_reduce(part, G, B, f->d, y, ex, st);
@@ -2731,6 +2288,26 @@ asf_status ffn_t(const asf_ffn *f, const void *x, int B, const int32_t *idx, con
   return cuda_status(e);
 }
 
+// The FFN rows of the descriptor's hot_rows leading neurons.
+HotBlock hot_block_of(const asf_ffn *f) {
+  HotBlock hb{};
+  const int rows = std::min(std::max(0, f->hot_rows), f->n);
+  if (rows == 0) return hb;
+  const size_t es = esize(f->wdtype);
+  if (ffn_packed(f)) {
+    hb.p[0] = static_cast<const unsigned char *>(f->act == ASF_ACT_REGLU ? f->Wg : f->Wu);
+    hb.bytes[0] = (long long)((size_t)rows * (size_t)ffn_rs(f) * es) & ~15ll;
+    return hb;
+  }
+  const void *mats[3] = {f->act == ASF_ACT_REGLU ? f->Wg : nullptr, f->Wu, f->WdT};
+  for (int i = 0; i < 3; ++i) {
+    if (!mats[i]) continue;
+    hb.p[i] = static_cast<const unsigned char *>(mats[i]);
+    hb.bytes[i] = (long long)(((size_t)(rows - 1) * (size_t)ffn_rs(f) + (size_t)f->d) * es) & ~15ll;
+  }
+  return hb;
+}
+
 // One layer, predictor then sparse FFN.  Workspace: header | predictor
 // scratch (mask, h) | FFN scratch.  When layer 2 leaves the union mask and the
 // fused FFN can rank it, no compaction kernel runs: the FFN kernel builds its
@@ -2749,7 +2326,8 @@ asf_status predict_ffn_t(const asf_predictor *p, const asf_ffn *f, const void *x
   unsigned char *fs = base + kHeaderBytes + pred_scratch(p, B);
   bool mask_only = pred_leaves_mask<T>(p, B);
   if (parts & kPartPredict) {
-    if (predict_layers<T>(p, x, B, thr, idx, count, hdr, mask, h, st, mask_only) != cudaSuccess) return ASF_ERR_CUDA;
+    if (predict_layers<T>(p, x, B, thr, idx, count, hdr, mask, h, st, mask_only, hot_block_of(f)) != cudaSuccess)
+      return ASF_ERR_CUDA;
   }
   if (!(parts & kPartFfn)) return ASF_OK;
   Exchange ex;

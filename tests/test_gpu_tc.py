@@ -1,8 +1,9 @@
-"""The many-token path on the tensor cores (fp16 weights, B > 4 for the FFN,
-B > 8 for predictor layer 2) against the oracle: list lengths across the
-activation-chunk (32) and MMA-tile (128) boundaries, empty lists, ragged d
-and n, every token-padding class (N = 16, 32, 64), and the predictor's
-index lists bit-exact on conditioned inputs."""
+"""The many-token path (fp16 weights, B > 4): gate/up on the tensor cores in
+launches of 16 tokens, the down projection on the CUDA cores, against the
+oracle: list lengths across the ownership-chunk (32) and MMA-tile (128)
+boundaries, empty lists, ragged d and n, one and two token launches (B <= 16
+and B <= 32), and the predictor's index lists at those batch sizes bit-exact
+on conditioned inputs."""
 import numpy as np
 import pytest
 import torch

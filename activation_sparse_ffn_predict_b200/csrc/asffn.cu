@@ -2027,16 +2027,18 @@ cudaError_t pred2_reg_any(const asf_predictor *p, int B, float thr, const float 
 // fits the ring); otherwise the register-streaming kernel compacts itself.
 template <typename T>
 bool pred_leaves_mask(const asf_predictor *p, int B) {
-  if (B > 8 || n_words_of(p->n) > kCompactThreads * kCompactWords) return false;
+  if (n_words_of(p->n) > kCompactThreads * kCompactWords) return false;
   const int sms = sm_count();
   const int rpc = (p->n + sms - 1) / sms;
   int CR, NSL;
-  return ring_shape((size_t)p->r * sizeof(T), pred2_vec_bytes(nb_cover(B), p->r, rpc), kRing2Budget, rpc, CR, NSL);
+  return ring_shape((size_t)p->r * sizeof(T), pred2_vec_bytes(nb_cover(std::min(B, 8)), p->r, rpc), kRing2Budget,
+                    rpc, CR, NSL);
 }
 
 // Layer 1 (register-streaming kernel, token groups of up to 8), then layer 2:
-// batches of up to 8 tokens use the bulk-copy ring kernel followed by the
-// compaction kernel when the slice fits; larger batches use the
+// the bulk-copy ring kernel, once per group of up to 8 tokens -- the union is
+// an OR over tokens, so every group ORs into the same mask -- followed by the
+// compaction kernel, when the slice fits the ring; otherwise the
 // register-streaming layer-2 kernel, which compacts in its last CTA.
 template <typename T>
 cudaError_t predict_layers(const asf_predictor *p, const void *x, int B, float thr, int32_t *idx, int32_t *count,
@@ -2046,9 +2048,12 @@ cudaError_t predict_layers(const asf_predictor *p, const void *x, int B, float t
   cudaError_t e = pred1_reg_any<T>(p, x, B, h, mask, st);
   if (e != cudaSuccess) return e;
   if (mask_only) {
-    bool used = false;
-    e = pred2_ring_any<T>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
-    if (e == cudaSuccess && !used) e = cudaErrorInvalidConfiguration;   // pred_leaves_mask said it fits
+    for (int g0 = 0; g0 < B && e == cudaSuccess; g0 += 8) {
+      bool used = false;
+      e = pred2_ring_any<T>(p, std::min(8, B - g0), thr, h + (size_t)g0 * p->r, mask, idx, count, hdr, st, used,
+                            g0 == 0 ? hot : HotBlock());
+      if (e == cudaSuccess && !used) e = cudaErrorInvalidConfiguration;   // pred_leaves_mask said it fits
+    }
     return e;
   }
   return pred2_reg_any<T>(p, B, thr, h, mask, idx, count, hdr, st);

@@ -45,19 +45,27 @@ class LayerStack:
         self.graph: Optional[torch.cuda.CUDAGraph] = None
 
     def launches_per_step(self) -> int:
-        """Kernels this library launches per step, following its dispatch: the
-        predictor is two GEMV kernels plus the compaction kernel for batches
-        of up to 8 tokens (the register-streaming layer-2 kernel compacts
-        itself above that); the sparse or dense FFN is two kernels.  In the
-        combined call the fused sparse FFN (batches up to 4 whose per-lane
-        accumulators fit) ranks the mask itself and no compaction runs."""
+        """Kernels this library launches per step, following its dispatch.
+        Predictor: the layer-1 kernel, the layer-2 ring kernel once per group
+        of up to 8 tokens (all groups OR into one union mask), and the
+        compaction kernel -- except in the combined call when the one-kernel
+        sparse FFN (batches up to 4 whose per-lane accumulators fit) ranks the
+        mask itself.  FFN: the one-kernel FFN and its reduction (B <= 4); for
+        larger batches with fp16 weights the tensor-core gate/up kernel once
+        per 16 tokens and the down projection; otherwise gate/up and down on
+        the CUDA cores."""
+        fused = _fused_sparse_ffn(self.d, self.dtype, self.B)
+        if fused:
+            ffn = 2
+        elif self.dtype == torch.float16:
+            ffn = -(-self.B // 16) + 1
+        else:
+            ffn = 2
         if self.mode != "predict":
-            return self.L * 2
-        if self.B > 8:
-            return self.L * 4
-        if self.combined and _fused_sparse_ffn(self.d, self.dtype, self.B):
-            return self.L * 4
-        return self.L * 5
+            return self.L * ffn
+        pred = 1 + -(-self.B // 8)
+        compact = 0 if (self.combined and fused) else 1
+        return self.L * (pred + compact + ffn)
 
     def enqueue(self, stream=None) -> None:
         for l in range(self.L):

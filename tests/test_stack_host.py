@@ -25,14 +25,19 @@ class _Stub:
         self.d, self.dtype, self.B, self.L, self.mode, self.combined = d, dtype, B, L, mode, combined
 
 
-@pytest.mark.parametrize("B,mode,combined,per_layer", [
-    (1, "predict", True, 4),    # layer 1, layer 2 ring, sparse FFN ranking the mask, reduction
-    (1, "predict", False, 5),   # + the compaction kernel between the two calls
-    (4, "predict", True, 4),
-    (6, "predict", True, 5),    # ring layer 2 + compaction, two-kernel FFN
-    (12, "predict", True, 4),   # register layer 2 compacts itself, two-kernel FFN
-    (1, "sparse", True, 2), (32, "dense", True, 2),
+@pytest.mark.parametrize("B,dtype,mode,combined,per_layer", [
+    (1, torch.float16, "predict", True, 4),    # layer 1, layer 2 ring, sparse FFN ranking the mask, reduction
+    (1, torch.float16, "predict", False, 5),   # + the compaction kernel between the two calls
+    (4, torch.float16, "predict", True, 4),
+    (6, torch.float16, "predict", True, 5),    # ring + compaction, tensor-core gate/up + down
+    (12, torch.float16, "predict", True, 6),   # two ring groups of tokens
+    (16, torch.float16, "predict", True, 6),
+    (17, torch.float16, "predict", True, 8),   # three ring groups, two gate/up launches
+    (32, torch.float16, "predict", True, 9),   # four ring groups, two gate/up launches
+    (12, torch.float32, "predict", True, 6),   # fp32: CUDA-core gate/up + down
+    (1, torch.float16, "sparse", True, 2), (32, torch.float16, "dense", True, 3),
+    (32, torch.float32, "dense", True, 2),
 ])
-def test_launches_per_step(B, mode, combined, per_layer):
-    st = _Stub(4096, torch.float16, B, 32, mode, combined)
+def test_launches_per_step(B, dtype, mode, combined, per_layer):
+    st = _Stub(4096 if dtype == torch.float16 else 512, dtype, B, 32, mode, combined)
     assert ST.LayerStack.launches_per_step(st) == 32 * per_layer

@@ -230,25 +230,27 @@ def asf_predict_sparse_ffn_exchange(pred: Predictor, ffn: FFN, x: torch.Tensor, 
     check(st, "asf_predict_sparse_ffn_exchange")
 
 
-def asf_reduce_exchange(part: torch.Tensor, group, y: torch.Tensor, ws: Workspace, local_ranks: int = 1,
-                        stream=None) -> None:
+def asf_reduce_exchange(part: torch.Tensor, group, y: torch.Tensor, ws: Workspace, stream=None) -> None:
     """y = sum over ranks (rank order) of each rank's sum of its partials.
 
-    part: [G, B, d] fp32 (this rank's), or [world, G, B, d] with local_ranks ==
-    world (one process holding every rank, all run in one cooperative launch);
-    y: [B, d] or [world, B, d] accordingly."""
-    if local_ranks == 1:
-        if part.dim() != 3 or y.shape != part.shape[1:]:
-            raise ValueError("part must be [G, B, d] and y [B, d]")
+    part: [G, B, d] fp32, this rank's partials, with y [B, d]; or
+    [R, G, B, d] with y [R, B, d]: one process holding all R ranks of the
+    group (R = its world), run as one cooperative launch."""
+    if part.dim() == 3:
+        if y.shape != part.shape[1:]:
+            raise ValueError("part [G, B, d] needs y [B, d]")
+        local = 1
         G, B, d = part.shape
         prs, yrs = 0, 0
-    else:
-        if part.dim() != 4 or part.shape[0] != local_ranks or y.shape != (local_ranks,) + tuple(part.shape[2:]):
-            raise ValueError("part must be [world, G, B, d] and y [world, B, d]")
-        _, G, B, d = part.shape
+    elif part.dim() == 4:
+        local, G, B, d = part.shape
+        if y.shape != (local, B, d):
+            raise ValueError("part [R, G, B, d] needs y [R, B, d]")
         prs, yrs = G * B * d, B * d
+    else:
+        raise ValueError("part must be [G, B, d] or [R, G, B, d]")
     st = L.load().asf_reduce_exchange(_dev(part, "part", torch.float32), prs, int(G), int(B), int(d),
-                                      ctypes.byref(group), int(local_ranks), _dev(y, "y", torch.float32), yrs,
+                                      ctypes.byref(group), int(local), _dev(y, "y", torch.float32), yrs,
                                       ws.ptr, ws.nbytes, _stream(stream))
     check(st, "asf_reduce_exchange")
 

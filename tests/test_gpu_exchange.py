@@ -40,7 +40,7 @@ def test_emulated_exchange_sums_every_rank(world, G, B, d):
     for call in range(3):                          # consecutive calls alternate the halves
         part = torch.randn(world, G, B, d, device="cuda", generator=gen)
         y = torch.full((world, B, d), float("nan"), device="cuda")
-        A.asf_reduce_exchange(part, grp.desc, y, ws, local_ranks=world)
+        A.asf_reduce_exchange(part, grp.desc, y, ws)
         torch.cuda.synchronize()
         ref = part.double().sum(dim=(0, 1)).cpu().numpy()
         for r in range(world):
@@ -59,13 +59,13 @@ def test_missing_peer_times_out():
     ws = _ws()
     part = torch.randn(G, B, d, device="cuda")
     y = torch.zeros(B, d, device="cuda")
-    A.asf_reduce_exchange(part, grp.desc, y, ws, local_ranks=1)
+    A.asf_reduce_exchange(part, grp.desc, y, ws)
     torch.cuda.synchronize()
     assert A.asf_read_error(ws) == L.ASF_ERR_TIMEOUT
     assert rel_err(y.cpu().numpy(), part.double().sum(dim=0).cpu().numpy()) <= 1e-5
     # the device still works
     grp1 = SH.EmulatedGroup(1, d, max_batch=1)
-    A.asf_reduce_exchange(part, grp1.desc, y, ws, local_ranks=1)
+    A.asf_reduce_exchange(part, grp1.desc, y, ws)
     torch.cuda.synchronize()
     assert A.asf_read_error(ws) == 0
 

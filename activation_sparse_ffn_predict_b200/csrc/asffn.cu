@@ -944,7 +944,8 @@ template <int NT, bool REGLU>
 __global__ void __launch_bounds__(9 * kWarp)
     k_gu_tc(const __half *__restrict__ Wg, const __half *__restrict__ Wu, const float *__restrict__ bias,
             const __half *__restrict__ x, int d, long long rs, int n, int B, const int32_t *__restrict__ idx,
-            const int32_t *__restrict__ count, float *__restrict__ a, int Btot, int g0, Header *__restrict__ hdr) {
+            const int32_t *__restrict__ count, float *__restrict__ a, __half *__restrict__ a2, int Btot, int g0,
+            Header *__restrict__ hdr) {
   using Lg = GuTc<NT, REGLU>;
   constexpr int NS = Lg::NS;
   constexpr int MATS = REGLU ? 2 : 1;
@@ -1128,7 +1129,28 @@ __global__ void __launch_bounds__(9 * kWarp)
       }
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
-      if (!owned || j >= cnt) continue;
+      if (!owned) continue;
+      if (a2) {
+        // the down kernel's operand: for chunk q of 32 positions and token
+        // group gg of 8, rows 0-7 hold fp16(a) of the group's tokens and rows
+        // 8-15 fp16(a - fp16(a)); positions past the list and padding tokens
+        // are zero (the down kernel reads whole chunks and groups)
+        const int q = j / kTcChunk, ngt = (Btot + 7) / 8;
+#pragma unroll
+        for (int b = 0; b < NT; ++b) {
+          const int t = g0 + b;
+          if (t >= 8 * ngt) break;
+          float v = 0.f;
+          if (got && k >= 0 && j < cnt && b < B) v = REGLU ? fmaxf(g[b] + bk, 0.f) * u[b] : fmaxf(u[b] + bk, 0.f);
+          const __half hi = __float2half_rn(v);
+          const __half lo = __float2half_rn(v - __half2float(hi));
+          __half *dst = a2 + (((size_t)q * ngt + (t >> 3)) * 16 + (t & 7)) * kTcChunk + lane;
+          dst[0] = hi;
+          dst[8 * kTcChunk] = lo;
+        }
+        continue;
+      }
+      if (j >= cnt) continue;
 #pragma unroll
       for (int b = 0; b < NT; ++b) {
         if (b >= B) break;
@@ -1143,6 +1165,222 @@ __global__ void __launch_bounds__(9 * kWarp)
   if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tbase, Lg::COLS);
+  }
+}
+
+// Down projection of a batch on the tensor cores: y = sum_k a_k WdT[k] over
+// the list, as D[col][n] = sum_k WdT[k][col] a2[n][k] with the activations
+// carried as fp16 hi/lo pairs (hi = fp16(a), lo = fp16(a - hi): together a to
+// about 2^-22 relative, so the sum stays as close to fp32 as on the CUDA
+// cores).  Work item w = (column range r of 128, list split s) of an R x S
+// grid of items; CTA c takes items c, c + G, ... .  Per item, the stages are
+// the split's chunks of 32 positions: the W_down^T tile [32 neurons][128
+// columns] (MN-major, 128-byte swizzle: the 8-neuron group kg and 64-column
+// atom at (2 kg + atom) * 1024) and, per group of 8 tokens, the a2 tile [16
+// rows][32] (K-major, 64-byte swizzle, 1 KB).  One thread issues, per stage,
+// 2 K-steps x NG groups of M 128 x N 16 x K 16 MMAs into the 16-column
+// accumulator of each group (64 tensor-memory columns in all); warps 0-3 read
+// an item's accumulators (lane = column), add hi and lo and write the item's
+// partial y[s][b][col]; k_reduce_partials sums the S splits in order.
+template <int NG>
+struct DnTc {
+  static constexpr int W = kTcChunk * kTcRows * 2;     // 8 KB
+  static constexpr int A = NG * 16 * kTcChunk * 2;     // NG KB
+  static constexpr int STAGE = W + A;
+  static constexpr int NS = 8;
+  static constexpr int BAR = 1024;
+  static constexpr size_t SMEM = 1024 + BAR + (size_t)NS * STAGE;
+  static constexpr uint32_t COLS = 64;
+  static_assert(STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+  static_assert(NG * 16 <= (int)COLS, "one 16-column accumulator per token group");
+};
+
+template <int NG>
+__global__ void __launch_bounds__(9 * kWarp)
+    k_down_tc(const __half *__restrict__ WdT, const __half *__restrict__ a2, const int32_t *__restrict__ idx,
+              const int32_t *__restrict__ count, int d, long long rs, int n, int B, int R, int S,
+              float *__restrict__ part, Header *__restrict__ hdr) {
+  using Ld = DnTc<NG>;
+  constexpr int NS = Ld::NS;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = align1024(smem_raw);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *empty = full + NS;
+  uint64_t *tfull = empty + NS;
+  uint64_t *tempty = tfull + 1;
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(tempty + 1);
+  unsigned char *stages = smem + Ld::BAR;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t *err = &hdr->err;
+
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < NS; ++q) {
+      mbar_init(&full[q], 4 * kWarp);
+      mbar_init(&empty[q], 1);
+    }
+    mbar_init(&tfull[0], 1);
+    mbar_init(&tempty[0], 4 * kWarp);
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tslot, Ld::COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  pdl_wait();
+  pdl_trigger();
+
+  int cnt = n;
+  if (idx) cnt = max(0, min(ld_cg_i32(count), n));
+  const int nch = (cnt + kTcChunk - 1) / kTcChunk;
+  const int items = R * S;
+  // chunks of item w: the s-th of S equal shares of the list
+  auto item_chunks = [&](int w, int &q0) {
+    const int sp = w / R;
+    q0 = (int)((long long)nch * sp / S);
+    return (int)((long long)nch * (sp + 1) / S) - q0;
+  };
+
+  if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ producers --
+    const int t = threadIdx.x - 4 * kWarp;
+    const int kn = t >> 2, quarter = t & 3;         // neuron of the chunk, quarter of its 256-byte segment
+    const uint64_t pol = l2_evict_first();
+    bool ok = true;
+    int it = 0;                                      // stages issued so far (all items)
+    for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
+      const int col0 = (w % R) * kTcRows;
+      int q0;
+      const int nq = item_chunks(w, q0);
+      for (int qi = 0; qi < nq; ++qi, ++it) {
+        const int sl = it % NS;
+        if (it >= NS && !mbar_wait(&empty[sl], (uint32_t)((it / NS) - 1) & 1u, kWaitNs)) {
+          flag_error(err, kErrTimeout);
+          ok = false;
+          break;
+        }
+        unsigned char *st = stages + (size_t)sl * Ld::STAGE;
+        const int q = q0 + qi;
+        const int j = q * kTcChunk + kn;
+        int k = -1;
+        if (j < cnt) {
+          k = idx ? ld_cg_i32(idx + j) : j;
+          if ((unsigned)k >= (unsigned)n) k = -1;   // flagged by the gate/up kernel
+        }
+        const __half *rowp = WdT + (size_t)max(k, 0) * rs;
+        unsigned char *wt = st + (size_t)(kn >> 3) * 2048 + (size_t)(kn & 7) * 128;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int ci = quarter * 4 + cc;             // 16-byte chunk of the 256-byte segment
+          const int col = col0 + ci * 8;
+          const bool in = k >= 0 && col < d;
+          cp_async16(wt + (size_t)(ci >> 3) * 1024 + (((ci & 7) ^ (kn & 7)) << 4),
+                     in ? (const void *)(rowp + col) : (const void *)WdT, in ? 16u : 0u, pol);
+        }
+        unsigned char *at = st + Ld::W;
+        for (int qq = t; qq < NG * 16 * 4; qq += 4 * kWarp) {
+          const int row = qq >> 2, c = qq & 3;       // row 16 g + r of the NG group tiles
+          cp_async16(at + (size_t)(row >> 4) * 1024 + (row & 15) * 64 + ((c ^ (((row & 15) >> 1) & 3)) << 4),
+                     a2 + (((size_t)q * NG + (row >> 4)) * 16 + (row & 15)) * kTcChunk + c * 8, 16u);
+        }
+        cp_async_commit();
+        if (it >= NS - 1) {
+          cp_async_wait<NS - 1>();
+          fence_proxy_async_smem();
+          mbar_arrive(&full[(it - (NS - 1)) % NS]);
+        }
+      }
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    if (ok)
+      for (int e = max(0, it - (NS - 1)); e < it; ++e) mbar_arrive(&full[e % NS]);
+  } else if (warp == 8) {
+    // ------------------------------------------------------------------ MMA --
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_f16(kTcRows, kTcN, 1, 0);
+      bool ok = true;
+      int it = 0, done = 0;                          // stages consumed, items with accumulators
+      for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
+        int q0;
+        const int nq = item_chunks(w, q0);
+        if (nq == 0) continue;
+        if (done >= 1 && !mbar_wait(&tempty[0], (uint32_t)(done - 1) & 1u, kWaitNs)) {
+          flag_error(err, kErrTimeout);
+          break;
+        }
+        tc_fence_after();
+        for (int qi = 0; qi < nq; ++qi, ++it) {
+          const int sl = it % NS;
+          if (!mbar_wait(&full[sl], (uint32_t)(it / NS) & 1u, kWaitNs)) {
+            flag_error(err, kErrTimeout);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          unsigned char *st = stages + (size_t)sl * Ld::STAGE;
+#pragma unroll
+          for (int kk = 0; kk < kTcChunk / 16; ++kk) {
+            // neurons 16 kk .. 16 kk + 15: 8-neuron groups 2 kk, 2 kk + 1 (SBO 2048); columns: atoms 0, 1 (LBO 1024)
+            const uint64_t ad = umma_desc(st + (size_t)(2 * kk) * 2048, 1024, 2048, kSwz128);
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+              const uint64_t bd = umma_desc(st + Ld::W + g * 1024 + kk * 32, 16, 512, kSwz64);
+              umma_f16(tbase + (uint32_t)(kTcN * g), ad, bd, idesc, (qi | kk) != 0);
+            }
+          }
+          umma_commit(&empty[sl]);
+        }
+        if (ok) umma_commit(&tfull[0]);
+        ++done;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- epilogue --
+    const uint32_t lane_addr = tbase + ((uint32_t)(kWarp * warp) << 16);
+    int done = 0;
+    for (int w = blockIdx.x; w < items; w += gridDim.x) {
+      int q0;
+      const int nq = item_chunks(w, q0);
+      const int col = (w % R) * kTcRows + kWarp * warp + lane;
+      const int sp = w / R;
+      bool got = false;
+      if (nq > 0) {
+        got = __all_sync(0xffffffffu, mbar_wait(&tfull[0], (uint32_t)done & 1u, kWaitNs));
+        if (!got && lane == 0) flag_error(err, kErrTimeout);
+        tc_fence_after();
+      }
+      float v[NG][16];
+      __syncwarp();          // tensor-memory loads below are warp-synchronous
+      if (got) {
+#pragma unroll
+        for (int g = 0; g < NG; ++g) tmem_ld16(lane_addr + (uint32_t)(kTcN * g), v[g]);
+      }
+      if (nq > 0) {
+        tc_fence_before();
+        mbar_arrive(&tempty[0]);
+        ++done;
+      }
+      if (col < d) {
+#pragma unroll
+        for (int g = 0; g < NG; ++g)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int b = 8 * g + e;
+            if (b < B) part[((size_t)sp * B + b) * d + col] = got ? v[g][e] + v[g][8 + e] : 0.f;
+          }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Ld::COLS);
   }
 }
 
@@ -1868,10 +2106,36 @@ bool ffn_packed(const asf_ffn *f) {
 
 size_t pred_scratch(const asf_predictor *p, int B) { return mask_region(p) + r256((size_t)B * p->r * 4); }
 
+// Tensor-core down projection: column ranges of 128 and list splits chosen so
+// that the R x S work items fill whole waves of CTAs (at least 95% busy when
+// some S <= 32 allows it).
+int tc_ranges(const asf_ffn *f) { return (f->d + kTcRows - 1) / kTcRows; }
+int tc_splits(const asf_ffn *f) {
+  const int R = tc_ranges(f), G = std::min(sm_count(), kMaxGrid);
+  int best = 1;
+  double best_eff = -1.0;
+  for (int S = 1; S <= 32; ++S) {
+    const int items = R * S;
+    const int ctas = std::min(G, items);
+    const double eff = (double)items / ((double)((items + ctas - 1) / ctas) * ctas);
+    if (eff >= 0.95) return S;
+    if (eff > best_eff) {
+      best_eff = eff;
+      best = S;
+    }
+  }
+  return best;
+}
+int tc_groups(int B) { return (B + 7) / 8; }
+size_t tc_a2_bytes(const asf_ffn *f, int B) {
+  return r256((size_t)((f->n + kTcChunk - 1) / kTcChunk) * tc_groups(B) * 16 * kTcChunk * 2);
+}
+
 size_t ffn_scratch(const asf_ffn *f, int B) {
   const size_t two_kernel = r256((size_t)f->n * B * 4) + r256((size_t)down_splits(f) * B * f->d * 4);
   const size_t fused = r256((size_t)std::min(sm_count(), kMaxGrid) * B * f->d * 4);
-  return std::max(two_kernel, fused);
+  const size_t tc = f->wdtype == ASF_F16 && B > 4 ? tc_a2_bytes(f, B) + r256((size_t)tc_splits(f) * B * f->d * 4) : 0;
+  return std::max({two_kernel, fused, tc});
 }
 
 asf_status check_pred(const asf_predictor *p) {
@@ -2130,34 +2394,49 @@ cudaError_t launch_final_reduce(const float *part, int G, int B, int d, float *y
 
 // ------------------------------------------------------ tensor-core ffn --
 // B in 5..32 with fp16 weights: gate/up on tcgen05 in launches of 16 tokens
-// (one pass over the rows for B <= 16, two for B <= 32), then the down
-// projection over the same list on the CUDA cores.
+// (one pass over the rows for B <= 16, two for B <= 32) writing the
+// activations as fp16 hi/lo pairs, then the down projection on tcgen05 over
+// the same list, and the fixed-order sum of its list splits.
 bool tc_ok(const asf_ffn *f, int B) { return f->wdtype == ASF_F16 && B > 4 && B <= ASF_MAX_BATCH; }
 
 template <bool REGLU>
 cudaError_t launch_gu_tc(const asf_ffn *f, const __half *x, int Bh, int Btot, int g0, const int32_t *idx,
-                         const int32_t *count, float *a, Header *hdr, cudaStream_t st) {
+                         const int32_t *count, float *a, __half *a2, Header *hdr, cudaStream_t st) {
   return launch(k_gu_tc<kTcN, REGLU>, dim3(std::min(sm_count(), kMaxGrid)), dim3(9 * kWarp),
                 GuTc<kTcN, REGLU>::SMEM, st, (const __half *)f->Wg, (const __half *)f->Wu, f->bias, x, f->d,
-                ffn_rs(f), f->n, Bh, idx, count, a, Btot, g0, hdr);
+                ffn_rs(f), f->n, Bh, idx, count, a, a2, Btot, g0, hdr);
+}
+
+template <int NG>
+cudaError_t launch_down_tc(const asf_ffn *f, int B, const int32_t *idx, const int32_t *count, const __half *a2,
+                           float *part, Header *hdr, cudaStream_t st) {
+  const int R = tc_ranges(f), S = tc_splits(f);
+  const int grid = std::min(std::min(sm_count(), kMaxGrid), R * S);
+  return launch(k_down_tc<NG>, dim3(grid), dim3(9 * kWarp), DnTc<NG>::SMEM, st, (const __half *)f->WdT, a2, idx,
+                count, f->d, ffn_rs(f), f->n, B, R, S, part, hdr);
 }
 
 cudaError_t run_tc(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *y,
                    Header *hdr, unsigned char *scratch, cudaStream_t st, const Exchange &ex) {
-  float *a = reinterpret_cast<float *>(scratch);
-  float *part = reinterpret_cast<float *>(scratch + r256((size_t)f->n * B * 4));
+  __half *a2 = reinterpret_cast<__half *>(scratch);
+  float *part = reinterpret_cast<float *>(scratch + tc_a2_bytes(f, B));
   const bool reglu = f->act == ASF_ACT_REGLU;
   cudaError_t e = cudaSuccess;
   for (int g0 = 0; g0 < B && e == cudaSuccess; g0 += kTcN) {
     const int Bh = std::min(kTcN, B - g0);
     const __half *xg = static_cast<const __half *>(x) + (size_t)g0 * f->d;
-    e = reglu ? launch_gu_tc<true>(f, xg, Bh, B, g0, idx, count, a, hdr, st)
-              : launch_gu_tc<false>(f, xg, Bh, B, g0, idx, count, a, hdr, st);
+    e = reglu ? launch_gu_tc<true>(f, xg, Bh, B, g0, idx, count, nullptr, a2, hdr, st)
+              : launch_gu_tc<false>(f, xg, Bh, B, g0, idx, count, nullptr, a2, hdr, st);
   }
   if (e != cudaSuccess) return e;
-  e = run_down<__half, 8>(f, B, idx, count, a, part, y, hdr, st);
-  if (e == cudaSuccess && ex.grp) e = launch_final_reduce(y, 1, B, f->d, y, ex, st);
-  return e;
+  switch (tc_groups(B)) {
+    case 1: e = launch_down_tc<1>(f, B, idx, count, a2, part, hdr, st); break;
+    case 2: e = launch_down_tc<2>(f, B, idx, count, a2, part, hdr, st); break;
+    case 3: e = launch_down_tc<3>(f, B, idx, count, a2, part, hdr, st); break;
+    default: e = launch_down_tc<4>(f, B, idx, count, a2, part, hdr, st); break;
+  }
+  if (e != cudaSuccess) return e;
+  return launch_final_reduce(part, tc_splits(f), B, f->d, y, ex, st);
 }
 
 // ------------------------------------------------------------- fused ffn --

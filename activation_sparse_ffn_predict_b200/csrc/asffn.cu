@@ -2134,7 +2134,7 @@ size_t tc_a2_bytes(const asf_ffn *f, int B) {
 size_t ffn_scratch(const asf_ffn *f, int B) {
   const size_t two_kernel = r256((size_t)f->n * B * 4) + r256((size_t)down_splits(f) * B * f->d * 4);
   const size_t fused = r256((size_t)std::min(sm_count(), kMaxGrid) * B * f->d * 4);
-  const size_t tc = f->wdtype == ASF_F16 && B > 4 ? tc_a2_bytes(f, B) + r256((size_t)tc_splits(f) * B * f->d * 4) : 0;
+  const size_t tc = f->wdtype == ASF_F16 ? tc_a2_bytes(f, B) + r256((size_t)tc_splits(f) * B * f->d * 4) : 0;
   return std::max({two_kernel, fused, tc});
 }
 
@@ -2393,11 +2393,15 @@ cudaError_t launch_final_reduce(const float *part, int G, int B, int d, float *y
 }
 
 // ------------------------------------------------------ tensor-core ffn --
-// B in 5..32 with fp16 weights: gate/up on tcgen05 in launches of 16 tokens
+// fp16 batches the one-kernel FFN cannot hold (B > 4, or too many per-lane
+// accumulators at a wide d): gate/up on tcgen05 in launches of 16 tokens
 // (one pass over the rows for B <= 16, two for B <= 32) writing the
 // activations as fp16 hi/lo pairs, then the down projection on tcgen05 over
 // the same list, and the fixed-order sum of its list splits.
-bool tc_ok(const asf_ffn *f, int B) { return f->wdtype == ASF_F16 && B > 4 && B <= ASF_MAX_BATCH; }
+bool fused_ok(const asf_ffn *f, int B);
+bool tc_ok(const asf_ffn *f, int B) {
+  return f->wdtype == ASF_F16 && B >= 1 && B <= ASF_MAX_BATCH && !fused_ok(f, B);
+}
 
 template <bool REGLU>
 cudaError_t launch_gu_tc(const asf_ffn *f, const __half *x, int Bh, int Btot, int g0, const int32_t *idx,

@@ -29,13 +29,13 @@ class _Stub:
     (1, torch.float16, "predict", True, 4),    # layer 1, layer 2 ring, sparse FFN ranking the mask, reduction
     (1, torch.float16, "predict", False, 5),   # + the compaction kernel between the two calls
     (4, torch.float16, "predict", True, 4),
-    (6, torch.float16, "predict", True, 5),    # ring + compaction, tensor-core gate/up + down
-    (12, torch.float16, "predict", True, 6),   # two ring groups of tokens
-    (16, torch.float16, "predict", True, 6),
-    (17, torch.float16, "predict", True, 8),   # three ring groups, two gate/up launches
-    (32, torch.float16, "predict", True, 9),   # four ring groups, two gate/up launches
+    (6, torch.float16, "predict", True, 6),    # ring + compaction, tensor-core gate/up, down, reduction
+    (12, torch.float16, "predict", True, 7),   # two ring groups of tokens
+    (16, torch.float16, "predict", True, 7),
+    (17, torch.float16, "predict", True, 9),   # three ring groups, two gate/up launches
+    (32, torch.float16, "predict", True, 10),  # four ring groups, two gate/up launches
     (12, torch.float32, "predict", True, 6),   # fp32: CUDA-core gate/up + down
-    (1, torch.float16, "sparse", True, 2), (32, torch.float16, "dense", True, 3),
+    (1, torch.float16, "sparse", True, 2), (32, torch.float16, "dense", True, 4),
     (32, torch.float32, "dense", True, 2),
 ])
 def test_launches_per_step(B, dtype, mode, combined, per_layer):

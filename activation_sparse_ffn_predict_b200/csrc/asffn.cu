@@ -543,10 +543,7 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
   if (warp == kRingWarps && lane == 0) {
     for (int i = 0; i < min(nch, NSL); ++i) ring_issue(W2, r, row0, row1, CR, NSL, i, ring, full);
   }
-  // The FFN rows of the hot block (active for most tokens) go to L2 now, while
-  // the predictor's own streams leave HBM bandwidth idle; the sparse FFN that
-  // follows then gathers its active hot rows from L2.
-  if (warp == kRingWarps) prefetch_hot(hot, blockIdx.x, gridDim.x);
+
   // biases are weights too: fetched before the wait, read from shared memory
   // (the consumers' named barrier below orders these stores)
   if (warp < kRingWarps)
@@ -556,6 +553,14 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
   if (warp == kRingWarps) {
     if (lane == 0 && !ring_produce(W2, r, row0, row1, CR, NSL, NSL, nch, ring, full, empty))
       flag_error(&hdr->err, kErrTimeout);
+    // Every W2 copy of this CTA is queued: the FFN rows of the hot block
+    // (active for most tokens) now go to L2, in the window where HBM idles
+    // between this kernel's last copies and the sparse FFN's first, which
+    // then gathers its active hot rows from L2.  (Issued at this kernel's
+    // start instead, the prefetch competed with the W2 stream and measured
+    // slower.)
+    __syncwarp();
+    prefetch_hot(hot, blockIdx.x, gridDim.x);
   } else {
     {
       // 4 consecutive floats of h land together in one plane (r % 8 == 0 for

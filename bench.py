@@ -48,9 +48,10 @@ def parse_args(argv=None):
     p.add_argument("--no-hot-perm", action="store_true", help="keep neuron id order")
     p.add_argument("--layout", choices=["packed", "split"], default="packed",
                    help="FFN weight layout: neuron-major packed rows, or separate W_gate/W_up/W_down^T")
-    p.add_argument("--hot-prefetch", action="store_true",
-                   help="pass the hot-row prefetch hint to the sparse FFN (off by default: the rows it "
-                        "warms that the list then skips cost more than the warm-up saves)")
+    p.add_argument("--no-hot-prefetch", action="store_true",
+                   help="with hot rows first, do not pass the hot-block hint (asf_ffn.hot_rows: the rows "
+                        "active for at least half of the calibration tokens, pulled into L2 by the "
+                        "predictor's layer-2 kernel once its W2 copies are queued)")
     p.add_argument("--l2-next", action="store_true",
                    help="let each sparse FFN prefetch the next layer's predictor weights into L2 (off by "
                         "default: the stack measured faster without it)")
@@ -279,7 +280,7 @@ def workload_config(cfg, args):
             "l2": "inputs larger than L2: every step streams rows of all layers of a stack "
                   "whose weights exceed the 126 MB L2 many times over",
             "l2_next": (args.mode == "predict" and args.l2_next),
-            "hot_row_hint": bool(args.hot_prefetch),
+            "hot_row_hint": bool(hot and not args.no_hot_prefetch),
             "parallelism": f"replicas x{args.gpus}"}
 
 
@@ -363,7 +364,7 @@ def run_ours(args, cfg):
         if hot:
             w, share, hr = hot_permute_layer(cfg, l, w, device)
             shares.append(share)
-            hr = hr if args.hot_prefetch else 0
+            hr = 0 if args.no_hot_prefetch else hr
             hot_rows.append(hr)
         preds.append(Predictor(w.W1, w.b1, w.W2, w.b2))
         if args.layout == "packed":

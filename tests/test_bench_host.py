@@ -65,4 +65,4 @@ def test_default_command_line(bench):
     assert a.gpus == 1 and a.batch == 1 and a.mode == "predict" and a.impl == "ours"
     assert a.warmup >= 3 and a.steps >= 1
     assert a.config == "llama70b_reglu" and a.layout == "packed"     # the largest single-GPU stack
-    assert not a.hot_prefetch and not a.l2_next
+    assert not a.no_hot_prefetch and not a.l2_next      # hot-block hint on where rows are hot-first

@@ -1003,19 +1003,26 @@ __global__ void __launch_bounds__(9 * kWarp)
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ producers --
-    const int t = threadIdx.x - 4 * kWarp;        // tile row of this thread
+    // Thread t copies 16-byte chunk c = t % 8 of tile rows t / 8 + 16 i: the 8
+    // threads of a row read its 128 bytes together, so one warp instruction
+    // covers four whole lines.
+    const int t = threadIdx.x - 4 * kWarp;
+    const int c = t & 7, rsub = t >> 3;
     const uint64_t pol = l2_evict_first();
     const __half *mats[2] = {REGLU ? Wg : Wu, Wu};
-    int krow = -1;
+    int krow[kTcRows / 16];
     bool ok = true;
     for (int it = 0; it < total && ok; ++it) {
       const int T = it / nK, kc = it - T * nK, sl = it % NS;
       if (kc == 0) {
-        const int j = own0 + T * kTcRows + t;
-        krow = -1;
-        if (j < own1 && j < cnt) {
-          const int k = idx ? ld_cg_i32(idx + j) : j;
-          if ((unsigned)k < (unsigned)n) krow = k;
+#pragma unroll
+        for (int i = 0; i < kTcRows / 16; ++i) {
+          const int j = own0 + T * kTcRows + rsub + 16 * i;
+          krow[i] = -1;
+          if (j < own1 && j < cnt) {
+            const int k = idx ? ld_cg_i32(idx + j) : j;
+            if ((unsigned)k < (unsigned)n) krow[i] = k;
+          }
         }
       }
       if (it >= NS && !mbar_wait(&empty[sl], (uint32_t)((it / NS) - 1) & 1u, kWaitNs)) {
@@ -1025,23 +1032,24 @@ __global__ void __launch_bounds__(9 * kWarp)
       }
       unsigned char *st = stages + (size_t)sl * Lg::STAGE;
       const int col0 = kc * kTcK;
+      const bool cin = col0 + c * 8 < d;
 #pragma unroll
       for (int m = 0; m < MATS; ++m) {
-        const __half *rowp = mats[m] + (size_t)max(krow, 0) * rs + col0;
-        unsigned char *dt = st + (size_t)m * Lg::W + (size_t)t * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const bool in = krow >= 0 && col0 + c * 8 < d;
-          cp_async16(dt + ((c ^ (t & 7)) << 4), in ? (const void *)(rowp + c * 8) : (const void *)mats[m],
-                     in ? 16u : 0u, pol);
+        for (int i = 0; i < kTcRows / 16; ++i) {
+          const int rr = rsub + 16 * i;
+          const bool in = krow[i] >= 0 && cin;
+          const __half *src = mats[m] + (size_t)max(krow[i], 0) * rs + col0 + c * 8;
+          cp_async16(st + (size_t)m * Lg::W + (size_t)rr * 128 + ((c ^ (rr & 7)) << 4),
+                     in ? (const void *)src : (const void *)mats[m], in ? 16u : 0u, pol);
         }
       }
       unsigned char *xt = st + (size_t)MATS * Lg::W;
       for (int q = t; q < NT * 8; q += 4 * kWarp) {
-        const int b = q >> 3, c = q & 7;
-        const bool in = b < B && col0 + c * 8 < d;
-        cp_async16(xt + b * 128 + ((c ^ (b & 7)) << 4),
-                   in ? (const void *)(x + (size_t)b * d + col0 + c * 8) : (const void *)x, in ? 16u : 0u);
+        const int b = q >> 3, cx = q & 7;
+        const bool in = b < B && col0 + cx * 8 < d;
+        cp_async16(xt + b * 128 + ((cx ^ (b & 7)) << 4),
+                   in ? (const void *)(x + (size_t)b * d + col0 + cx * 8) : (const void *)x, in ? 16u : 0u);
       }
       cp_async_commit();
       if (it >= NS - 1) {
@@ -1251,8 +1259,11 @@ __global__ void __launch_bounds__(9 * kWarp)
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ producers --
+    // Thread t copies 16-byte chunk ci = t % 16 of the 256-byte row segments
+    // of neurons t / 16 + 8 i: 16 threads read a segment together, so one warp
+    // instruction covers two whole segments.
     const int t = threadIdx.x - 4 * kWarp;
-    const int kn = t >> 2, quarter = t & 3;         // neuron of the chunk, quarter of its 256-byte segment
+    const int ci = t & 15, nsub = t >> 4;
     const uint64_t pol = l2_evict_first();
     bool ok = true;
     int it = 0;                                      // stages issued so far (all items)
@@ -1269,21 +1280,20 @@ __global__ void __launch_bounds__(9 * kWarp)
         }
         unsigned char *st = stages + (size_t)sl * Ld::STAGE;
         const int q = q0 + qi;
-        const int j = q * kTcChunk + kn;
-        int k = -1;
-        if (j < cnt) {
-          k = idx ? ld_cg_i32(idx + j) : j;
-          if ((unsigned)k >= (unsigned)n) k = -1;   // flagged by the gate/up kernel
-        }
-        const __half *rowp = WdT + (size_t)max(k, 0) * rs;
-        unsigned char *wt = st + (size_t)(kn >> 3) * 2048 + (size_t)(kn & 7) * 128;
+        const int col = col0 + ci * 8;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int ci = quarter * 4 + cc;             // 16-byte chunk of the 256-byte segment
-          const int col = col0 + ci * 8;
+        for (int i = 0; i < kTcChunk / 8; ++i) {
+          const int kn = nsub + 8 * i;
+          const int j = q * kTcChunk + kn;
+          int k = -1;
+          if (j < cnt) {
+            k = idx ? ld_cg_i32(idx + j) : j;
+            if ((unsigned)k >= (unsigned)n) k = -1;   // flagged by the gate/up kernel
+          }
           const bool in = k >= 0 && col < d;
-          cp_async16(wt + (size_t)(ci >> 3) * 1024 + (((ci & 7) ^ (kn & 7)) << 4),
-                     in ? (const void *)(rowp + col) : (const void *)WdT, in ? 16u : 0u, pol);
+          cp_async16(st + (size_t)(kn >> 3) * 2048 + (size_t)(ci >> 3) * 1024 + (size_t)(kn & 7) * 128 +
+                         (((ci & 7) ^ (kn & 7)) << 4),
+                     in ? (const void *)(WdT + (size_t)k * rs + col) : (const void *)WdT, in ? 16u : 0u, pol);
         }
         unsigned char *at = st + Ld::W;
         for (int qq = t; qq < NG * 16 * 4; qq += 4 * kWarp) {

@@ -1003,26 +1003,19 @@ __global__ void __launch_bounds__(9 * kWarp)
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ producers --
-    // Thread t copies 16-byte chunk c = t % 8 of tile rows t / 8 + 16 i: the 8
-    // threads of a row read its 128 bytes together, so one warp instruction
-    // covers four whole lines.
-    const int t = threadIdx.x - 4 * kWarp;
-    const int c = t & 7, rsub = t >> 3;
+    const int t = threadIdx.x - 4 * kWarp;        // tile row of this thread
     const uint64_t pol = l2_evict_first();
     const __half *mats[2] = {REGLU ? Wg : Wu, Wu};
-    int krow[kTcRows / 16];
+    int krow = -1;
     bool ok = true;
     for (int it = 0; it < total && ok; ++it) {
       const int T = it / nK, kc = it - T * nK, sl = it % NS;
       if (kc == 0) {
-#pragma unroll
-        for (int i = 0; i < kTcRows / 16; ++i) {
-          const int j = own0 + T * kTcRows + rsub + 16 * i;
-          krow[i] = -1;
-          if (j < own1 && j < cnt) {
-            const int k = idx ? ld_cg_i32(idx + j) : j;
-            if ((unsigned)k < (unsigned)n) krow[i] = k;
-          }
+        const int j = own0 + T * kTcRows + t;
+        krow = -1;
+        if (j < own1 && j < cnt) {
+          const int k = idx ? ld_cg_i32(idx + j) : j;
+          if ((unsigned)k < (unsigned)n) krow = k;
         }
       }
       if (it >= NS && !mbar_wait(&empty[sl], (uint32_t)((it / NS) - 1) & 1u, kWaitNs)) {
@@ -1032,24 +1025,23 @@ __global__ void __launch_bounds__(9 * kWarp)
       }
       unsigned char *st = stages + (size_t)sl * Lg::STAGE;
       const int col0 = kc * kTcK;
-      const bool cin = col0 + c * 8 < d;
 #pragma unroll
       for (int m = 0; m < MATS; ++m) {
+        const __half *rowp = mats[m] + (size_t)max(krow, 0) * rs + col0;
+        unsigned char *dt = st + (size_t)m * Lg::W + (size_t)t * 128;
 #pragma unroll
-        for (int i = 0; i < kTcRows / 16; ++i) {
-          const int rr = rsub + 16 * i;
-          const bool in = krow[i] >= 0 && cin;
-          const __half *src = mats[m] + (size_t)max(krow[i], 0) * rs + col0 + c * 8;
-          cp_async16(st + (size_t)m * Lg::W + (size_t)rr * 128 + ((c ^ (rr & 7)) << 4),
-                     in ? (const void *)src : (const void *)mats[m], in ? 16u : 0u, pol);
+        for (int c = 0; c < 8; ++c) {
+          const bool in = krow >= 0 && col0 + c * 8 < d;
+          cp_async16(dt + ((c ^ (t & 7)) << 4), in ? (const void *)(rowp + c * 8) : (const void *)mats[m],
+                     in ? 16u : 0u, pol);
         }
       }
       unsigned char *xt = st + (size_t)MATS * Lg::W;
       for (int q = t; q < NT * 8; q += 4 * kWarp) {
-        const int b = q >> 3, cx = q & 7;
-        const bool in = b < B && col0 + cx * 8 < d;
-        cp_async16(xt + b * 128 + ((cx ^ (b & 7)) << 4),
-                   in ? (const void *)(x + (size_t)b * d + col0 + cx * 8) : (const void *)x, in ? 16u : 0u);
+        const int b = q >> 3, c = q & 7;
+        const bool in = b < B && col0 + c * 8 < d;
+        cp_async16(xt + b * 128 + ((c ^ (b & 7)) << 4),
+                   in ? (const void *)(x + (size_t)b * d + col0 + c * 8) : (const void *)x, in ? 16u : 0u);
       }
       cp_async_commit();
       if (it >= NS - 1) {
@@ -1259,11 +1251,8 @@ __global__ void __launch_bounds__(9 * kWarp)
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ producers --
-    // Thread t copies 16-byte chunk ci = t % 16 of the 256-byte row segments
-    // of neurons t / 16 + 8 i: 16 threads read a segment together, so one warp
-    // instruction covers two whole segments.
     const int t = threadIdx.x - 4 * kWarp;
-    const int ci = t & 15, nsub = t >> 4;
+    const int kn = t >> 2, quarter = t & 3;         // neuron of the chunk, quarter of its 256-byte segment
     const uint64_t pol = l2_evict_first();
     bool ok = true;
     int it = 0;                                      // stages issued so far (all items)
@@ -1280,20 +1269,21 @@ __global__ void __launch_bounds__(9 * kWarp)
         }
         unsigned char *st = stages + (size_t)sl * Ld::STAGE;
         const int q = q0 + qi;
-        const int col = col0 + ci * 8;
+        const int j = q * kTcChunk + kn;
+        int k = -1;
+        if (j < cnt) {
+          k = idx ? ld_cg_i32(idx + j) : j;
+          if ((unsigned)k >= (unsigned)n) k = -1;   // flagged by the gate/up kernel
+        }
+        const __half *rowp = WdT + (size_t)max(k, 0) * rs;
+        unsigned char *wt = st + (size_t)(kn >> 3) * 2048 + (size_t)(kn & 7) * 128;
 #pragma unroll
-        for (int i = 0; i < kTcChunk / 8; ++i) {
-          const int kn = nsub + 8 * i;
-          const int j = q * kTcChunk + kn;
-          int k = -1;
-          if (j < cnt) {
-            k = idx ? ld_cg_i32(idx + j) : j;
-            if ((unsigned)k >= (unsigned)n) k = -1;   // flagged by the gate/up kernel
-          }
+        for (int cc = 0; cc < 4; ++cc) {
+          const int ci = quarter * 4 + cc;             // 16-byte chunk of the 256-byte segment
+          const int col = col0 + ci * 8;
           const bool in = k >= 0 && col < d;
-          cp_async16(st + (size_t)(kn >> 3) * 2048 + (size_t)(ci >> 3) * 1024 + (size_t)(kn & 7) * 128 +
-                         (((ci & 7) ^ (kn & 7)) << 4),
-                     in ? (const void *)(WdT + (size_t)k * rs + col) : (const void *)WdT, in ? 16u : 0u, pol);
+          cp_async16(wt + (size_t)(ci >> 3) * 1024 + (((ci & 7) ^ (kn & 7)) << 4),
+                     in ? (const void *)(rowp + col) : (const void *)WdT, in ? 16u : 0u, pol);
         }
         unsigned char *at = st + Ld::W;
         for (int qq = t; qq < NG * 16 * 4; qq += 4 * kWarp) {
@@ -2125,14 +2115,16 @@ size_t pred_scratch(const asf_predictor *p, int B) { return mask_region(p) + r25
 // that the R x S work items fill whole waves of CTAs (at least 95% busy when
 // some S <= 32 allows it).
 int tc_ranges(const asf_ffn *f) { return (f->d + kTcRows - 1) / kTcRows; }
+// List splits S of the tensor-core down projection: the fewest whose R x S
+// equal work items fill whole waves of one CTA per SM to at least 95% (R = 64
+// column ranges at d = 8192 alone would leave 84 of 148 SMs idle).
 int tc_splits(const asf_ffn *f) {
   const int R = tc_ranges(f), G = std::min(sm_count(), kMaxGrid);
   int best = 1;
   double best_eff = -1.0;
   for (int S = 1; S <= 32; ++S) {
     const int items = R * S;
-    const int ctas = std::min(G, items);
-    const double eff = (double)items / ((double)((items + ctas - 1) / ctas) * ctas);
+    const double eff = (double)items / ((double)((items + G - 1) / G) * G);
     if (eff >= 0.95) return S;
     if (eff > best_eff) {
       best_eff = eff;
@@ -2146,10 +2138,12 @@ size_t tc_a2_bytes(const asf_ffn *f, int B) {
   return r256((size_t)((f->n + kTcChunk - 1) / kTcChunk) * tc_groups(B) * 16 * kTcChunk * 2);
 }
 
+bool tc_ok(const asf_ffn *f, int B);
+
 size_t ffn_scratch(const asf_ffn *f, int B) {
   const size_t two_kernel = r256((size_t)f->n * B * 4) + r256((size_t)down_splits(f) * B * f->d * 4);
   const size_t fused = r256((size_t)std::min(sm_count(), kMaxGrid) * B * f->d * 4);
-  const size_t tc = f->wdtype == ASF_F16 ? tc_a2_bytes(f, B) + r256((size_t)tc_splits(f) * B * f->d * 4) : 0;
+  const size_t tc = tc_ok(f, B) ? tc_a2_bytes(f, B) + r256((size_t)tc_splits(f) * B * f->d * 4) : 0;
   return std::max({two_kernel, fused, tc});
 }
 
@@ -2280,9 +2274,20 @@ cudaError_t pred2_ring_any(const asf_predictor *p, int B, float thr, const float
   }
 }
 
+// Token groups of layer 1: up to 8 tokens of x staged at once.  A batch of 8
+// or more tokens may use 200 KB of shared memory for them (its FFN is not the
+// one-kernel FFN, which this kernel has to fit beside), so a batch of 16 reads
+// W1 twice, not four times, at d = 8192 and 12288.
+int pred1_nb(int B, size_t bytes_per_token) {
+  int nb = 8;
+  const size_t budget = B >= 8 ? 200 * 1024 : kSmemBudget;
+  while (nb > 1 && (nb > B || (size_t)nb * bytes_per_token > budget)) nb >>= 1;
+  return nb;
+}
+
 template <typename T>
 cudaError_t pred1_reg_any(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, cudaStream_t st) {
-  switch (pick_nb(B, (size_t)p->d * sizeof(T))) {
+  switch (pred1_nb(B, (size_t)p->d * sizeof(T))) {
     case 1: return run_pred_l1<T, 1>(p, x, B, h, mask, st);
     case 2: return run_pred_l1<T, 2>(p, x, B, h, mask, st);
     case 4: return run_pred_l1<T, 4>(p, x, B, h, mask, st);
@@ -2408,15 +2413,14 @@ cudaError_t launch_final_reduce(const float *part, int G, int B, int d, float *y
 }
 
 // ------------------------------------------------------ tensor-core ffn --
-// fp16 batches the one-kernel FFN cannot hold (B > 4, or too many per-lane
-// accumulators at a wide d): gate/up on tcgen05 in launches of 16 tokens
+// fp16 batches of 5..32 tokens: gate/up on tcgen05 in launches of 16 tokens
 // (one pass over the rows for B <= 16, two for B <= 32) writing the
 // activations as fp16 hi/lo pairs, then the down projection on tcgen05 over
-// the same list, and the fixed-order sum of its list splits.
-bool fused_ok(const asf_ffn *f, int B);
-bool tc_ok(const asf_ffn *f, int B) {
-  return f->wdtype == ASF_F16 && B >= 1 && B <= ASF_MAX_BATCH && !fused_ok(f, B);
-}
+// the same list, and the fixed-order sum of its list splits.  Batches of up
+// to 4 the one-kernel FFN cannot hold (B >= 3 at d = 8192) stay on the CUDA
+// cores: a 16-token MMA tile would be at most a quarter used, and the
+// CUDA-core pair measured about twice as fast there.
+bool tc_ok(const asf_ffn *f, int B) { return f->wdtype == ASF_F16 && B > 4 && B <= ASF_MAX_BATCH; }
 
 template <bool REGLU>
 cudaError_t launch_gu_tc(const asf_ffn *f, const __half *x, int Bh, int Btot, int g0, const int32_t *idx,

@@ -51,13 +51,14 @@ class LayerStack:
         compaction kernel -- except in the combined call when the one-kernel
         sparse FFN (batches up to 4 whose per-lane accumulators fit) ranks the
         mask itself.  FFN: the one-kernel FFN and its reduction when it holds
-        the batch; otherwise with fp16 weights the tensor-core gate/up kernel
-        once per 16 tokens, the tensor-core down projection and the reduction
-        of its splits; with fp32 weights gate/up and down on the CUDA cores."""
+        the batch; otherwise, for 5-32 tokens with fp16 weights, the
+        tensor-core gate/up kernel once per 16 tokens, the tensor-core down
+        projection and the reduction of its splits; else gate/up and down on
+        the CUDA cores."""
         fused = _fused_sparse_ffn(self.d, self.dtype, self.B)
         if fused:
             ffn = 2
-        elif self.dtype == torch.float16:
+        elif self.dtype == torch.float16 and self.B > 4:
             ffn = -(-self.B // 16) + 2
         else:
             ffn = 2

@@ -41,3 +41,15 @@ class _Stub:
 def test_launches_per_step(B, dtype, mode, combined, per_layer):
     st = _Stub(4096 if dtype == torch.float16 else 512, dtype, B, 32, mode, combined)
     assert ST.LayerStack.launches_per_step(st) == 32 * per_layer
+
+
+@pytest.mark.parametrize("d,B,per_layer", [
+    (8192, 1, 4),    # the one-kernel FFN holds one token at d = 8192
+    (8192, 2, 4),
+    (8192, 4, 5),    # too many accumulators: compaction + CUDA-core gate/up and down
+    (12288, 2, 5),
+    (12288, 6, 6),   # tensor-core gate/up, down, reduction
+])
+def test_launches_per_step_wide_layers(d, B, per_layer):
+    st = _Stub(d, torch.float16, B, 80, "predict", True)
+    assert ST.LayerStack.launches_per_step(st) == 80 * per_layer

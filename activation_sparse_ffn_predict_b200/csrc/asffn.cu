@@ -312,6 +312,101 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Layer 1 for rows too long to load into registers ahead of the wait (16 KB
+// and more at d >= 8192, fp16): the CTA's whole W1 slice goes to shared memory
+// in one bulk copy per row, issued at entry, before griddepcontrol.wait.  The
+// kernel then needs as much shared memory as the previous layer's sparse FFN
+// leaves free only once that kernel's CTAs exit, so its copies overlap the
+// FFN's tail and the reduction of its partials instead of following them.
+// After the wait it stages x one token group of NB at a time (the slice stays
+// in shared memory: W1 is read from HBM once for any batch), waits for each
+// row's copy (bounded), and warps take rows round-robin.
+constexpr int kPred1SmemRows = 16;    // most W1 rows one CTA stages
+template <typename T, int NB>
+__global__ void __launch_bounds__(kThreads)
+    k_pred_l1_smem(const T *__restrict__ W1, const float *__restrict__ b1, const T *__restrict__ x, int d,
+                   int r, int B, int rpc, float *__restrict__ h, uint32_t *__restrict__ mask_words, int n_words,
+                   int32_t *__restrict__ err) {
+  extern __shared__ __align__(128) unsigned char smem_p1[];
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem_p1);
+  T *ws = reinterpret_cast<T *>(smem_p1 + kPred1SmemRows * 8);
+  T *xs = ws + (size_t)rpc * d;
+  __shared__ int s_fail;
+  constexpr int V = Vec<T>::N;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row0 = blockIdx.x * rpc;
+  const int nrows = max(0, min(r, row0 + rpc) - row0);
+  const int nvec = d / V;
+  const uint32_t row_bytes = (uint32_t)((size_t)d * sizeof(T));
+  if (threadIdx.x == 0) {
+    s_fail = 0;
+    for (int i = 0; i < nrows; ++i) mbar_init(&bar[i], 1);
+    fence_mbar_init();
+    const uint64_t pol = l2_evict_first();
+    for (int i = 0; i < nrows; ++i) {
+      mbar_arrive_expect_tx(&bar[i], row_bytes);
+      bulk_g2s_stream(ws + (size_t)i * d, W1 + (size_t)(row0 + i) * d, row_bytes, &bar[i], pol);
+    }
+  }
+  // the biases of this warp's rows are weights too: loaded before the wait
+  float bias[kPred1SmemRows / kWarps];
+#pragma unroll
+  for (int j = 0; j < kPred1SmemRows / kWarps; ++j) {
+    const int i = warp + j * kWarps;
+    bias[j] = i < nrows ? __ldg(b1 + row0 + i) : 0.f;
+  }
+  pdl_trigger();
+  pdl_wait();
+  for (int w = blockIdx.x * kThreads + threadIdx.x; w < n_words; w += gridDim.x * kThreads) mask_words[w] = 0u;
+  bool ok = true;
+  for (int g0 = 0; g0 < B; g0 += NB) {
+    const int nb = min(NB, B - g0);
+    __syncthreads();      // also publishes the barrier initialisation (first group)
+    stage_tokens<T, NB>(xs, x, d, g0, nb);
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kPred1SmemRows / kWarps; ++j) {
+      const int i = warp + j * kWarps;
+      if (i >= nrows) break;
+      if (g0 == 0 && ok && !mbar_wait(&bar[i], 0u, kWaitNs)) {
+        if (lane == 0) flag_error(err, kErrTimeout);
+        ok = false;
+        s_fail = 1;
+      }
+      // two accumulators per token: the chunk pairs' products in separate chains
+      float acc[2][NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) acc[0][b] = acc[1][b] = 0.f;
+      if (ok) {
+        const T *wr = ws + (size_t)i * d;
+        for (int c0 = lane; c0 < nvec; c0 += 2 * kWarp) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = c0 + e * kWarp;
+            if (c < nvec) {
+              const uint4 wv = *reinterpret_cast<const uint4 *>(wr + (size_t)c * V);
+#pragma unroll
+              for (int b = 0; b < NB; ++b)
+                acc[e][b] = Vec<T>::dot(wv, *reinterpret_cast<const uint4 *>(xs + (size_t)b * d + (size_t)c * V),
+                                        acc[e][b]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float sum = warp_sum(acc[0][b] + acc[1][b]);
+        if (lane == b && b < nb) h[(size_t)(g0 + b) * r + row0 + i] = fmaxf(sum + bias[j], 0.f);
+      }
+    }
+  }
+  // a copy whose wait gave up may still be in flight: let it land (bounded)
+  // before the CTA's shared memory is released
+  __syncthreads();
+  if (s_fail && threadIdx.x == 0)
+    for (int i = 0; i < nrows; ++i) mbar_wait(&bar[i], 0u, kWaitNs);
+}
+
 // Stage h[g0..g0+nb) ([B][r] fp32) for dot products with rows of T.  For fp16
 // rows (8 elements per 16-byte chunk) the 8 floats of chunk c are split into
 // two planes of 4 so that a warp's shared-memory reads are conflict-free.
@@ -511,7 +606,7 @@ __host__ __device__ inline size_t pred2_vec_bytes(int NB, int r, int rpc) {
 // the bulk-copy ring (first chunks issued before the wait).  Each CTA ORs the
 // bits of its rows into the union mask; the next kernel compacts it.
 template <typename T, int NB>
-__global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
+__global__ void __launch_bounds__((kRingWarps + 1) * kWarp, 1)
     k_pred2_ring(const T *__restrict__ W2, const float *__restrict__ b2, const float *__restrict__ h, int r, int n,
                  int B, float thr, int rpc, int CR, int NSL, uint32_t *__restrict__ mask_words,
                  Header *__restrict__ hdr, HotBlock hot) {
@@ -630,36 +725,55 @@ __global__ void __launch_bounds__((kRingWarps + 1) * kWarp)
         ok = false;
       }
       const int ra = row0 + i * CR, rb = min(row1, ra + CR);
-      for (int row = ra + warp; row < rb && ok; row += kRingWarps) {
+      // two rows per pass (row and row + kRingWarps): their dot products and
+      // warp reductions are independent chains that overlap
+      for (int row = ra + warp; row < rb && ok; row += 2 * kRingWarps) {
+        const bool two = row + kRingWarps < rb;
         const T *wr = ring + ((size_t)sl * CR + (row - ra)) * r;
-        float acc[NB];
+        const T *wr2 = wr + (size_t)kRingWarps * r;
+        float acc[2][NB];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+        for (int b = 0; b < NB; ++b) acc[0][b] = acc[1][b] = 0.f;
         if (reg_h) {
 #pragma unroll
           for (int u = 0; u < HQ; ++u) {
             const int c = lane + u * kWarp;
             if (c < nvec) {
               const uint4 wv = *reinterpret_cast<const uint4 *>(wr + (size_t)c * V);
+              const uint4 wv2 = two ? *reinterpret_cast<const uint4 *>(wr2 + (size_t)c * V) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-              for (int b = 0; b < (kRegH ? NB : 1); ++b) acc[b] = Vec<T>::dotr(wv, hreg[b][u], acc[b]);
+              for (int b = 0; b < (kRegH ? NB : 1); ++b) {
+                acc[0][b] = Vec<T>::dotr(wv, hreg[b][u], acc[0][b]);
+                acc[1][b] = Vec<T>::dotr(wv2, hreg[b][u], acc[1][b]);
+              }
             }
           }
         } else {
           for (int c = lane; c < nvec; c += kWarp) {
             const uint4 wv = *reinterpret_cast<const uint4 *>(wr + (size_t)c * V);
+            const uint4 wv2 = two ? *reinterpret_cast<const uint4 *>(wr2 + (size_t)c * V) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-            for (int b = 0; b < NB; ++b) acc[b] += dot_hidden<T>(wv, hs + (size_t)b * r, r, c);
+            for (int b = 0; b < NB; ++b) {
+              acc[0][b] += dot_hidden<T>(wv, hs + (size_t)b * r, r, c);
+              acc[1][b] += dot_hidden<T>(wv2, hs + (size_t)b * r, r, c);
+            }
           }
         }
-        bool on = false;
+        bool on = false, on2 = false;
         const float bias = sb[row - row0];
+        const float bias2 = two ? sb[row + kRingWarps - row0] : 0.f;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          const float z = warp_sum(acc[b]) + bias;
+          const float z = warp_sum(acc[0][b]) + bias;
+          const float z2 = warp_sum(acc[1][b]) + bias2;
           on |= (b < B) && (z > thr);
+          on2 |= two && (b < B) && (z2 > thr);
         }
         if (lane == 0 && on) atomicOr(&smask[(row >> 5) - wfirst], 1u << (row & 31));
+        if (lane == 0 && on2) {
+          const int row2 = row + kRingWarps;
+          atomicOr(&smask[(row2 >> 5) - wfirst], 1u << (row2 & 31));
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[sl]);
@@ -1415,7 +1529,7 @@ __host__ __device__ inline FusedLayout fused_layout(int NS, int d, int M, int es
   o = align_up(o, 16);
   L.words = o; o += (size_t)(mask_words + 3) / 4 * 16 * 2;    // the words, then their prefix counts
   o = align_up(o, 16);
-  L.pd = o;    o += (size_t)kFusedWarps * L.grp * 2 * NB * 4;
+  L.pd = o;    o += (size_t)2 * kFusedWarps * L.grp * 2 * NB * 4;   // two buffers, alternate groups
   o = align_up(o, 128);
   L.x = o;     o += (size_t)NB * d * esz;
   o = align_up(o, 128);
@@ -1719,6 +1833,10 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     bool ok = true;
     for (int g0 = 0; g0 < nl; g0 += grp) {
       const int gn = min(grp, nl - g0);
+      // consecutive groups use alternate partial buffers: a warp writing the
+      // next group's partials has passed that group's barrier only after
+      // every warp has read this group's, so one barrier per group suffices
+      float *pdg = pd + (size_t)((g0 / grp) & 1) * (NW * grp * 2 * NB);
       for (int q = 0; q < gn; ++q) {
         const int i = g0 + q, s = i % NS;
         if (ok && !mbar_wait(&full[s], (uint32_t)(i / NS) & 1u, kWaitNs)) {
@@ -1755,8 +1873,8 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
         if (lane == 0) {
 #pragma unroll
           for (int b = 0; b < NB; ++b) {
-            pd[(((size_t)warp * grp + q) * 2 + 0) * NB + b] = pg[b];
-            pd[(((size_t)warp * grp + q) * 2 + 1) * NB + b] = pu[b];
+            pdg[(((size_t)warp * grp + q) * 2 + 0) * NB + b] = pg[b];
+            pdg[(((size_t)warp * grp + q) * 2 + 1) * NB + b] = pu[b];
           }
         }
       }
@@ -1770,8 +1888,8 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
           float g = 0.f, u = 0.f;
 #pragma unroll
           for (int w = 0; w < NW; ++w) {
-            g += pd[(((size_t)w * grp + q) * 2 + 0) * NB + b];
-            u += pd[(((size_t)w * grp + q) * 2 + 1) * NB + b];
+            g += pdg[(((size_t)w * grp + q) * 2 + 0) * NB + b];
+            u += pdg[(((size_t)w * grp + q) * 2 + 1) * NB + b];
           }
           float v = 0.f;
           if (k >= 0 && b < B) {
@@ -1798,7 +1916,6 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }
-      named_sync(1, NW * kWarp);
     }
     if (!ok) s_fail = 1;
   }
@@ -1830,38 +1947,64 @@ __global__ void __launch_bounds__((kFusedWarps + 1) * kWarp)
     for (int i = max(0, issued - NS); i < issued; ++i) mbar_wait(&full[i % NS], (uint32_t)(i / NS) & 1u, kWaitNs);
 }
 
-// y[b][col] = sum over the G per-CTA partials, in a fixed order: lanes own 32
-// consecutive columns (coalesced loads), the 8 warps split the partials and
-// all of a warp's loads are issued before any is added; warp sums are then
-// combined in warp order.
+// y[b][col] = sum over the G per-CTA partials, in a fixed order: a CTA owns
+// 32 * VEC consecutive columns (each lane VEC of them, loaded as one vector),
+// the 8 warps split the partials into runs of ceil(G / 8) and every warp sums
+// its run in order; warp sums are then combined in warp order (the same order
+// for every VEC).  The grid stays resident beside the sparse FFN from that
+// kernel's start, and the kernel stays small in registers, since at d = 4096
+// the next layer's layer-1 kernel must fit beside both: VEC 1 where that grid
+// fits one CTA per SM (128 CTAs at d = 4096), VEC 4 otherwise (64 CTAs at d =
+// 8192, 96 at 12288; 256 CTAs of VEC 1 there measured 3% slower end to end,
+// 128 of VEC 2 as slow).  part and y are 16-byte aligned and d % 4 == 0
+// (every caller's workspace and checked output).
 constexpr int kReduceWarps = 8;
-constexpr int kReduceMaxPerWarp = 32;   // G <= 256
+constexpr int kReduceMaxPerWarp = 32;      // G <= 256
+constexpr int kReduceBatch = 20;           // loads in flight per lane (G <= 160: one batch)
+
+template <int VEC> struct FVec;
+template <> struct FVec<1> { using type = float; };
+template <> struct FVec<4> { using type = float4; };
+__device__ __forceinline__ void fv_zero(float &a) { a = 0.f; }
+__device__ __forceinline__ void fv_zero(float4 &a) { a = make_float4(0.f, 0.f, 0.f, 0.f); }
+__device__ __forceinline__ void fv_add(float &a, float b) { a += b; }
+__device__ __forceinline__ void fv_add(float4 &a, float4 b) { a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w; }
+
+template <int VEC>
 __global__ void __launch_bounds__(kReduceWarps * kWarp)
     k_reduce_partials(const float *__restrict__ part, int G, int B, int d, float *__restrict__ y) {
-  __shared__ float red[kReduceWarps][kWarp];
+  using F = typename FVec<VEC>::type;
+  __shared__ F red[kReduceWarps][kWarp];
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int col = blockIdx.x * kWarp + lane;
+  const int col = (blockIdx.x * kWarp + lane) * VEC;
   const int b = blockIdx.y;
   const int per = (G + kReduceWarps - 1) / kReduceWarps;
   const int q0 = warp * per;
-  float v[kReduceMaxPerWarp];
+  F s;
+  fv_zero(s);
+  for (int u0 = 0; u0 < per; u0 += kReduceBatch) {
+    F v[kReduceBatch];
 #pragma unroll
-  for (int u = 0; u < kReduceMaxPerWarp; ++u) {
-    const int q = q0 + u;
-    v[u] = (u < per && q < G && col < d) ? ld_cg_f32(part + ((size_t)q * B + b) * d + col) : 0.f;
+    for (int u = 0; u < kReduceBatch; ++u) {
+      const int q = q0 + u0 + u;
+      if (u0 + u < per && q < G && col < d)
+        v[u] = __ldcg(reinterpret_cast<const F *>(part + ((size_t)q * B + b) * d + col));
+      else
+        fv_zero(v[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kReduceBatch; ++u) fv_add(s, v[u]);
   }
-  float s = 0.f;
-#pragma unroll
-  for (int u = 0; u < kReduceMaxPerWarp; ++u) s += v[u];
   red[warp][lane] = s;
   __syncthreads();
   if (warp == 0 && col < d) {
-    float t = 0.f;
+    F t;
+    fv_zero(t);
 #pragma unroll
-    for (int w = 0; w < kReduceWarps; ++w) t += red[w][lane];
-    y[(size_t)b * d + col] = t;
+    for (int w = 0; w < kReduceWarps; ++w) fv_add(t, red[w][lane]);
+    *reinterpret_cast<F *>(y + (size_t)b * d + col) = t;
   }
 }
 
@@ -2243,15 +2386,40 @@ bool ring_shape(size_t row_bytes, size_t vec_bytes, size_t budget, int rpc, int 
   return false;
 }
 
+// Ring of the layer-2 kernel.  Given the shared memory the layer-1 kernel
+// leaves free on an SM (beside > 0: layer 1 holds its W1 slice in shared
+// memory), three or more slots of at least 16 KB within it, so that the
+// layer-2 CTAs are resident, and their first W2 pieces in flight, while layer
+// 1 still runs; otherwise the 136 KB ring of 32 KB pieces, which becomes
+// resident as layer 1's CTAs exit.
+bool pred2_ring_shape(size_t row_bytes, size_t vec_bytes, size_t beside, int rpc, int &CR, int &NSL) {
+  const size_t fixed = ring_layout(8, 0, 1, 1, vec_bytes).total + 128;
+  if (beside > fixed) {
+    int cr = (int)std::min<size_t>(kRingChunk / row_bytes, (beside - fixed) / (3 * row_bytes));
+    cr = std::min(cr, std::max(1, rpc));
+    if (cr >= 1 && (size_t)cr * row_bytes >= 16 * 1024) {
+      const int chunks = (rpc + cr - 1) / cr;
+      for (int nsl = std::min(8, std::max(chunks, 2)); nsl >= 3; --nsl)
+        if (ring_layout(nsl, cr, 1, (int)row_bytes, vec_bytes).total <= beside) {
+          CR = cr;
+          NSL = nsl;
+          return true;
+        }
+    }
+  }
+  return ring_shape(row_bytes, vec_bytes, kRing2Budget, rpc, CR, NSL);
+}
+
 template <typename T, int NB>
 cudaError_t run_pred2_ring(const asf_predictor *p, int B, float thr, const float *h, uint32_t *mask, int32_t *idx,
-                           int32_t *count, Header *hdr, cudaStream_t st, bool &used, const HotBlock &hot) {
+                           int32_t *count, Header *hdr, cudaStream_t st, bool &used, const HotBlock &hot,
+                           size_t beside) {
   const int sms = sm_count();
   const int rpc = (p->n + sms - 1) / sms;
   const int grid = (p->n + rpc - 1) / rpc;
   const size_t vec = pred2_vec_bytes(NB, p->r, rpc);
   int CR, NSL;
-  used = ring_shape((size_t)p->r * sizeof(T), vec, kRing2Budget, rpc, CR, NSL);
+  used = pred2_ring_shape((size_t)p->r * sizeof(T), vec, beside, rpc, CR, NSL);
   if (!used) return cudaSuccess;
   const size_t smem = ring_layout(NSL, CR, p->r, (int)sizeof(T), vec).total;
   (void)idx;
@@ -2265,29 +2433,58 @@ inline int nb_cover(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 8; }
 
 template <typename T>
 cudaError_t pred2_ring_any(const asf_predictor *p, int B, float thr, const float *h, uint32_t *mask, int32_t *idx,
-                           int32_t *count, Header *hdr, cudaStream_t st, bool &used, const HotBlock &hot) {
+                           int32_t *count, Header *hdr, cudaStream_t st, bool &used, const HotBlock &hot,
+                           size_t beside) {
   switch (nb_cover(B)) {
-    case 1: return run_pred2_ring<T, 1>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
-    case 2: return run_pred2_ring<T, 2>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
-    case 4: return run_pred2_ring<T, 4>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
-    default: return run_pred2_ring<T, 8>(p, B, thr, h, mask, idx, count, hdr, st, used, hot);
+    case 1: return run_pred2_ring<T, 1>(p, B, thr, h, mask, idx, count, hdr, st, used, hot, beside);
+    case 2: return run_pred2_ring<T, 2>(p, B, thr, h, mask, idx, count, hdr, st, used, hot, beside);
+    case 4: return run_pred2_ring<T, 4>(p, B, thr, h, mask, idx, count, hdr, st, used, hot, beside);
+    default: return run_pred2_ring<T, 8>(p, B, thr, h, mask, idx, count, hdr, st, used, hot, beside);
   }
 }
 
-// Token groups of layer 1: up to 8 tokens of x staged at once.  A batch of 8
-// or more tokens may use 200 KB of shared memory for them (its FFN is not the
-// one-kernel FFN, which this kernel has to fit beside), so a batch of 16 reads
-// W1 twice, not four times, at d = 8192 and 12288.
-int pred1_nb(int B, size_t bytes_per_token) {
+// Shared memory of k_pred_l1_smem: the row barriers, the W1 slice of rpc
+// rows and NB tokens of x.
+constexpr size_t kPred1SmemMax = 226 * 1024;
+size_t pred1_smem_bytes(const asf_predictor *p, int rpc, int NB) {
+  return (size_t)kPred1SmemRows * 8 + ((size_t)rpc + NB) * p->d * esize(p->wdtype);
+}
+
+// Token group of layer 1 on the shared-memory slice kernel, or 0 when layer 1
+// stays on the register-streaming kernel: rows of at most 8 KB load into
+// registers before the wait there (a 16 x 16-byte chunk per lane), and that
+// kernel, 16 KB of shared memory at one token, sits beside the previous
+// layer's sparse FFN.
+int pred1_smem_nb(const asf_predictor *p, int B) {
+  const int sms = sm_count();
+  const int rpc = (p->r + sms - 1) / sms;
+  if (rpc > kPred1SmemRows || (size_t)p->d * esize(p->wdtype) <= 8192) return 0;
   int nb = 8;
-  const size_t budget = B >= 8 ? 200 * 1024 : kSmemBudget;
-  while (nb > 1 && (nb > B || (size_t)nb * bytes_per_token > budget)) nb >>= 1;
-  return nb;
+  while (nb > 1 && (nb > B || pred1_smem_bytes(p, rpc, nb) > kPred1SmemMax)) nb >>= 1;
+  return pred1_smem_bytes(p, rpc, nb) <= kPred1SmemMax ? nb : 0;
+}
+
+template <typename T, int NB>
+cudaError_t run_pred_l1_smem(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, int32_t *err,
+                             cudaStream_t st) {
+  const int sms = sm_count();
+  const int rpc = (p->r + sms - 1) / sms;
+  const int grid = (p->r + rpc - 1) / rpc;
+  return launch(k_pred_l1_smem<T, NB>, dim3(grid), dim3(kThreads), pred1_smem_bytes(p, rpc, NB), st,
+                (const T *)p->W1, p->b1, (const T *)x, p->d, p->r, B, rpc, h, mask, n_words_of(p->n), err);
 }
 
 template <typename T>
-cudaError_t pred1_reg_any(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, cudaStream_t st) {
-  switch (pred1_nb(B, (size_t)p->d * sizeof(T))) {
+cudaError_t pred1_reg_any(const asf_predictor *p, const void *x, int B, float *h, uint32_t *mask, int32_t *err,
+                          cudaStream_t st) {
+  switch (pred1_smem_nb(p, B)) {
+    case 1: return run_pred_l1_smem<T, 1>(p, x, B, h, mask, err, st);
+    case 2: return run_pred_l1_smem<T, 2>(p, x, B, h, mask, err, st);
+    case 4: return run_pred_l1_smem<T, 4>(p, x, B, h, mask, err, st);
+    case 8: return run_pred_l1_smem<T, 8>(p, x, B, h, mask, err, st);
+    default: break;
+  }
+  switch (pick_nb(B, (size_t)p->d * sizeof(T))) {
     case 1: return run_pred_l1<T, 1>(p, x, B, h, mask, st);
     case 2: return run_pred_l1<T, 2>(p, x, B, h, mask, st);
     case 4: return run_pred_l1<T, 4>(p, x, B, h, mask, st);
@@ -2319,6 +2516,20 @@ bool pred_leaves_mask(const asf_predictor *p, int B) {
                     rpc, CR, NSL);
 }
 
+constexpr size_t kSmSmem = 228 * 1024;        // shared memory of one SM
+constexpr size_t kCtaSmemReserve = 1024;      // the driver's share per resident CTA
+
+// Shared memory the layer-1 slice kernel of a batch of B leaves free on its SM
+// for the layer-2 ring (0 when layer 1 runs the register-streaming kernel).
+size_t pred2_beside_budget(const asf_predictor *p, int B) {
+  const int nb = pred1_smem_nb(p, B);
+  if (!nb) return 0;
+  const int sms = sm_count();
+  const int rpc1 = (p->r + sms - 1) / sms;
+  const size_t used = pred1_smem_bytes(p, rpc1, nb) + 256 + 2 * kCtaSmemReserve;   // + static, reserves
+  return used < kSmSmem ? kSmSmem - used : 0;
+}
+
 // Layer 1 (register-streaming kernel, token groups of up to 8), then layer 2:
 // the bulk-copy ring kernel, once per group of up to 8 tokens -- the union is
 // an OR over tokens, so every group ORs into the same mask -- followed by the
@@ -2329,13 +2540,14 @@ cudaError_t predict_layers(const asf_predictor *p, const void *x, int B, float t
                            Header *hdr, uint32_t *mask, float *h, cudaStream_t st, bool &mask_only,
                            const HotBlock &hot = HotBlock()) {
   mask_only = pred_leaves_mask<T>(p, B);
-  cudaError_t e = pred1_reg_any<T>(p, x, B, h, mask, st);
+  cudaError_t e = pred1_reg_any<T>(p, x, B, h, mask, &hdr->err, st);
   if (e != cudaSuccess) return e;
   if (mask_only) {
+    const size_t beside = pred2_beside_budget(p, B);
     for (int g0 = 0; g0 < B && e == cudaSuccess; g0 += 8) {
       bool used = false;
       e = pred2_ring_any<T>(p, std::min(8, B - g0), thr, h + (size_t)g0 * p->r, mask, idx, count, hdr, st, used,
-                            g0 == 0 ? hot : HotBlock());
+                            g0 == 0 ? hot : HotBlock(), beside);
       if (e == cudaSuccess && !used) e = cudaErrorInvalidConfiguration;   // pred_leaves_mask said it fits
     }
     return e;
@@ -2404,9 +2616,13 @@ PeerPtrs peer_ptrs(const asf_peer_group *g) {
 
 cudaError_t launch_final_reduce(const float *part, int G, int B, int d, float *y, const Exchange &ex,
                                 cudaStream_t st) {
-  if (!ex.grp)
-    return launch(k_reduce_partials, dim3((d + kWarp - 1) / kWarp, B), dim3(kReduceWarps * kWarp), 0, st, part, G, B,
-                  d, y);
+  if (!ex.grp) {
+    const int sms = sm_count();
+    const int vec = (long long)((d + kWarp - 1) / kWarp) * B <= sms ? 1 : 4;
+    const dim3 grid((d + kWarp * vec - 1) / (kWarp * vec), B);
+    if (vec == 1) return launch(k_reduce_partials<1>, grid, dim3(kReduceWarps * kWarp), 0, st, part, G, B, d, y);
+    return launch(k_reduce_partials<4>, grid, dim3(kReduceWarps * kWarp), 0, st, part, G, B, d, y);
+  }
   const asf_peer_group *g = ex.grp;
   return launch(k_reduce_exchange, dim3((d + kWarp - 1) / kWarp, B, 1), dim3(kReduceWarps * kWarp), 0, st, part,
                 0ll, G, B, d, (int)g->max_batch, peer_ptrs(g), g->epoch, y, 0ll, (int)g->world, (int)g->rank, ex.err);

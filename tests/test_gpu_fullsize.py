@@ -201,3 +201,50 @@ def test_fullsize_graph_stack_llama2_7b():
             assert rel_err(st.y[l].cpu().numpy(), yr) <= TOL[cfg.dtype]
     assert A.asf_read_error(st.ws) == 0
     st.release()
+
+
+@pytest.mark.parametrize("name", ["llama2_7b_reglu", "opt175b_relu"])
+def test_fullsize_packed_permuted_combined_stack(name):
+    """The benchmark's exact combination at full size: two layers permuted
+    hot-first through the library (activation counts, permutation, row
+    gather), packed neuron-major, with the hot-block hint, run as the captured
+    stack of combined calls; every layer's list bit-exact and its output within
+    tolerance of the oracle on the permuted weights."""
+    ensure_built()
+    import bench
+    from activation_sparse_ffn_predict_b200.api import FFN, Predictor, pack_layer
+    from activation_sparse_ffn_predict_b200.stack import LayerStack
+    cfg = S.get(name)
+    L = 2
+    preds, ffns, hosts, xs = [], [], [], []
+    for l in range(L):
+        w = S.layer_weights(cfg, l, device="cuda")
+        w, _, hot_rows = bench.hot_permute_layer(cfg, l, w, "cuda")
+        X = S.layer_tokens(cfg, l, 3, device="cuda")
+        W1, b1, W2 = w.W1.cpu().numpy(), w.b1.cpu().numpy(), w.W2.cpu().numpy()
+        b2 = condition_b2(W1, b1, W2, w.b2.cpu().numpy(), X.cpu().numpy(), cfg.tau)
+        w.b2 = torch.from_numpy(b2).cuda()
+        preds.append(Predictor(w.W1, w.b1, w.W2, w.b2))
+        ffns.append(FFN.packed(w.act, pack_layer(w.act, w.Wg, w.Wu, w.WdT), w.bias, hot_rows=hot_rows))
+        hosts.append((W1, b1, W2, b2, w))
+        xs.append(X)
+        assert hot_rows > 0
+    st = LayerStack(preds, ffns, 1, cfg.tau, mode="predict")
+    st.capture()
+    for t in range(2):
+        for l in range(L):
+            st.x[l].copy_(xs[l][t:t + 1])
+        st.step()
+        torch.cuda.synchronize()
+        for l in range(L):
+            W1, b1, W2, b2, w = hosts[l]
+            Xl = xs[l][t:t + 1].cpu().numpy()
+            ref = O.predict(W1, b1, W2, b2, Xl, cfg.tau)[0]
+            c = int(st.count[l].item())
+            np.testing.assert_array_equal(st.idx[l, :c].cpu().numpy(), ref)
+            g = torch.from_numpy(ref.astype(np.int64)).cuda()
+            take = lambda tt: None if tt is None else tt.index_select(0, g).cpu().numpy()
+            yr = O.sparse_ffn(w.act, take(w.Wg), take(w.Wu), take(w.WdT), take(w.bias), Xl, np.arange(ref.size))
+            assert rel_err(st.y[l].cpu().numpy(), yr) <= TOL[cfg.dtype]
+    assert A.asf_read_error(st.ws) == 0
+    st.release()

@@ -1377,6 +1377,31 @@ __global__ void __launch_bounds__(9 * kWarp)
     const int t = threadIdx.x - 4 * kWarp;
     const int kn = t >> 2, quarter = t & 3;         // neuron of the chunk, quarter of its 256-byte segment
     const uint64_t pol = l2_evict_first();
+    // The neuron of each stage is loaded four stages ahead (a ring of four
+    // registers): a stage's copies need its index, and loading it when the
+    // stage is issued exposed one L2 round trip per stage.  pw / pqi walk this
+    // CTA's stages in issue order (items w = blockIdx.x + G i that have
+    // chunks, their chunks in order); -1: no neuron.
+    int pw = blockIdx.x, pqi = 0, pq0 = 0, pnq = pw < items ? item_chunks(pw, pq0) : 0;
+    while (pw < items && pnq == 0) {
+      pw += gridDim.x;
+      pnq = pw < items ? item_chunks(pw, pq0) : 0;
+    }
+    auto next_index = [&]() {
+      int raw = -1;
+      if (pw < items) {
+        const int j = (pq0 + pqi) * kTcChunk + kn;
+        if (j < cnt) raw = idx ? ld_cg_i32(idx + j) : j;
+        ++pqi;
+        while (pw < items && pqi >= pnq) {
+          pw += gridDim.x;
+          pqi = 0;
+          pnq = pw < items ? item_chunks(pw, pq0) : 0;
+        }
+      }
+      return raw;
+    };
+    int kr0 = next_index(), kr1 = next_index(), kr2 = next_index(), kr3 = next_index();
     bool ok = true;
     int it = 0;                                      // stages issued so far (all items)
     for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
@@ -1392,12 +1417,12 @@ __global__ void __launch_bounds__(9 * kWarp)
         }
         unsigned char *st = stages + (size_t)sl * Ld::STAGE;
         const int q = q0 + qi;
-        const int j = q * kTcChunk + kn;
-        int k = -1;
-        if (j < cnt) {
-          k = idx ? ld_cg_i32(idx + j) : j;
-          if ((unsigned)k >= (unsigned)n) k = -1;   // flagged by the gate/up kernel
-        }
+        const int raw = kr0;
+        kr0 = kr1;
+        kr1 = kr2;
+        kr2 = kr3;
+        kr3 = next_index();
+        const int k = (unsigned)raw < (unsigned)n ? raw : -1;   // out of range: flagged by the gate/up kernel
         const __half *rowp = WdT + (size_t)max(k, 0) * rs;
         unsigned char *wt = st + (size_t)(kn >> 3) * 2048 + (size_t)(kn & 7) * 128;
 #pragma unroll

@@ -543,13 +543,20 @@ def run_ours(args, cfg):
     hbm_peak = float(peaks["hbm_gbs"])
     key = f"{cfg.name}:B{B}:{args.mode}"
     tr = traffic_record(key)
-    two = "k_sparse_ffn + k_reduce_partials" if B <= 4 else "k_compact + k_ffn_gu + k_ffn_down"
+    from activation_sparse_ffn_predict_b200.stack import _fused_sparse_ffn
+    if _fused_sparse_ffn(cfg.d, st.dtype, B):
+        two = "k_sparse_ffn + k_reduce_partials"
+    elif cfg.dtype == "f16" and B > 4:
+        two = "k_compact + k_gu_tc + k_down_tc + k_reduce_partials"
+    else:
+        two = "k_compact + k_ffn_gu + k_ffn_down"
     where = ("second half of asf_predict_sparse_ffn (asf_predict_sparse_ffn_end)" if args.mode == "predict"
              else f"asf_{args.mode}_ffn")
     roof = {"bound": "hbm", "kernel": f"{'dense' if args.mode == 'dense' else 'sparse'} FFN: {where} = {two}, "
                                       f"timed alone with CUDA events around it in a captured graph",
             "achieved": ffn_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": ffn_gbs / hbm_peak,
-            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+            "peak_source": ("measured: MEASURED_PEAKS.json hbm_gbs (burst copy)" if peak_src == "measured" else
+                            "fallback: 6650 GB/s from the profiling recipe (MEASURED_PEAKS.json absent)"),
             "frac_of_nominal_7700": ffn_gbs / NOMINAL_HBM_GBS,
             "traffic": traffic_per_launch(tr, ffn_bytes_prof / (nprof * L)),
             "traffic_source": (tr or {}).get("source"),

@@ -27,6 +27,7 @@
 // successor at entry.  Every wait on an mbarrier gives up after 200 ms and
 // records ASF_ERR_TIMEOUT in the workspace error word instead of hanging.
 
+#include <cuda.h>            // CUtensorMap and its encoder's types (the encoder comes from the runtime)
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -1069,11 +1070,12 @@ struct GuTc {
 // row), apply ReLU(g + b) * u (or ReLU(u + b)) and write a; two accumulator
 // buffers let the epilogue of one tile overlap the MMAs of the next.
 template <int NT, bool REGLU>
-__global__ void __launch_bounds__(9 * kWarp)
-    k_gu_tc(const __half *__restrict__ Wg, const __half *__restrict__ Wu, const float *__restrict__ bias,
-            const __half *__restrict__ x, int d, long long rs, int n, int B, const int32_t *__restrict__ idx,
-            const int32_t *__restrict__ count, float *__restrict__ a, __half *__restrict__ a2, int Btot, int g0,
-            Header *__restrict__ hdr) {
+__global__ void __launch_bounds__(9 * kWarp, 1)
+    k_gu_tc(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_u,
+            const __grid_constant__ CUtensorMap tm_x, int use_tma, const __half *__restrict__ Wg,
+            const __half *__restrict__ Wu, const float *__restrict__ bias, const __half *__restrict__ x, int d,
+            long long rs, int n, int B, const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
+            float *__restrict__ a, __half *__restrict__ a2, int Btot, int g0, Header *__restrict__ hdr) {
   using Lg = GuTc<NT, REGLU>;
   constexpr int NS = Lg::NS;
   constexpr int MATS = REGLU ? 2 : 1;
@@ -1088,9 +1090,10 @@ __global__ void __launch_bounds__(9 * kWarp)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t *err = &hdr->err;
 
+  __shared__ int srow[REGLU ? kTcRows : 1];    // the current tile's rows (TMA producers)
   if (threadIdx.x == 0) {
     for (int q = 0; q < NS; ++q) {
-      mbar_init(&full[q], 4 * kWarp);
+      mbar_init(&full[q], (REGLU && use_tma) ? 4 : 4 * kWarp);   // one arrival per producer warp / thread
       mbar_init(&empty[q], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -1124,8 +1127,74 @@ __global__ void __launch_bounds__(9 * kWarp)
   const int nK = (d + kTcK - 1) / kTcK;
   const int total = ntiles * nK;
 
-  if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ producers --
+  if (warp >= 4 && warp < 8 && REGLU && use_tma) {
+    // ------------------------------------------------ producers (gate + up) --
+    // TMA: warp 4 + p takes the four-row groups p, p + 4, ... of the tile,
+    // fetches their rows' indices, and its lane 0 issues, per stage, their
+    // gate and up rows as tile::gather4 loads
+    // (four rows of 64 columns per instruction; the maps' box is 64 columns x
+    // 1 row in the 128-byte swizzle, so the rows land in the layout the MMA
+    // reads), with warp 4 also loading x (a 2-D tile of 64 columns x 16
+    // tokens); each warp arrives on the stage once with its own bytes.
+    // Columns past d and tokens past B are outside the maps and read as
+    // zeros; groups of four rows wholly past the list are skipped, and other
+    // padding positions load row 0 (the epilogue writes zeros for them).
+    // Four issuing warps measured 19% faster (70B shape, B = 16) than the
+    // 16-byte cp.async gathers below, and one issuing thread 40% slower.
+    const int p = warp - 4;
+    const uint64_t pol = l2_evict_first();
+    bool ok = true;
+    int issued = 0;
+    int ng = 0;                      // this warp's four-row groups that hold listed positions
+    for (int it = 0; it < total && ok; ++it) {
+      const int T = it / nK, kc = it - T * nK, sl = it % NS;
+      if (kc == 0) {
+        // groups wholly past the list are not loaded: their accumulator rows
+        // are discarded by the epilogue, whatever the stage holds there
+        const int nvalid = min(kTcRows, max(0, min(own1, cnt) - (own0 + T * kTcRows)));
+        ng = min(8, max(0, ((nvalid + 3) / 4 - p + 3) / 4));    // groups p, p + 4, ... below nvalid
+        __syncwarp();
+        const int r = 4 * (p + 4 * (lane >> 2)) + (lane & 3);      // row 4g + e of group g = p + 4 (lane / 4)
+        const int j = own0 + T * kTcRows + r;
+        int k = 0;
+        if (j < own1 && j < cnt) {
+          const int kk = idx ? ld_cg_i32(idx + j) : j;
+          if ((unsigned)kk < (unsigned)n) k = kk;
+        }
+        srow[r] = k;
+        __syncwarp();
+      }
+      if (lane == 0) {
+        if (it >= NS && !mbar_wait(&empty[sl], (uint32_t)((it / NS) - 1) & 1u, kWaitNs)) {
+          flag_error(err, kErrTimeout);
+          ok = false;
+        } else {
+          unsigned char *st = stages + (size_t)sl * Lg::STAGE;
+          const int col0 = kc * kTcK;
+          mbar_arrive_expect_tx(&full[sl], (uint32_t)(ng * 2 * 512 + (p == 0 ? NT * kTcK * 2 : 0)));
+          for (int i = 0; i < ng; ++i) {
+            const int g = p + 4 * i;
+            tma_gather4(st + (size_t)g * 512, &tm_g, col0, srow[4 * g], srow[4 * g + 1], srow[4 * g + 2],
+                        srow[4 * g + 3], &full[sl], pol);
+            tma_gather4(st + (size_t)Lg::W + (size_t)g * 512, &tm_u, col0, srow[4 * g], srow[4 * g + 1],
+                        srow[4 * g + 2], srow[4 * g + 3], &full[sl], pol);
+          }
+          if (p == 0) tma_load_2d(st + (size_t)2 * Lg::W, &tm_x, col0, 0, &full[sl]);
+          issued = it + 1;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    // after a wait gave up, let each slot's last load land (bounded) before
+    // the shared memory is released
+    if (!ok && lane == 0)
+      for (int e = max(0, issued - NS); e < issued; ++e) mbar_wait(&full[e % NS], (uint32_t)(e / NS) & 1u, kWaitNs);
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------- producers (cp.async) --
+    // 16 bytes per thread, one tile row per thread.  Used for ReLU (one matrix
+    // per stage: the TMA gathers above measured 2% slower there) and for rows
+    // of up to 8 KB (d = 4096: a CTA's tile holds fewer listed rows there, and
+    // the TMA gathers measured 2-14% slower).
     const int t = threadIdx.x - 4 * kWarp;        // tile row of this thread
     const uint64_t pol = l2_evict_first();
     const __half *mats[2] = {REGLU ? Wg : Wu, Wu};
@@ -1325,8 +1394,8 @@ struct DnTc {
 
 template <int NG>
 __global__ void __launch_bounds__(9 * kWarp)
-    k_down_tc(const __half *__restrict__ WdT, const __half *__restrict__ a2, const int32_t *__restrict__ idx,
-              const int32_t *__restrict__ count, int d, long long rs, int n, int B, int R, int S,
+    k_down_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
+              const int32_t *__restrict__ idx, const int32_t *__restrict__ count, int d, int n, int B, int R, int S,
               float *__restrict__ part, Header *__restrict__ hdr) {
   using Ld = DnTc<NG>;
   constexpr int NS = Ld::NS;
@@ -1343,7 +1412,7 @@ __global__ void __launch_bounds__(9 * kWarp)
 
   if (threadIdx.x == 0) {
     for (int q = 0; q < NS; ++q) {
-      mbar_init(&full[q], 4 * kWarp);
+      mbar_init(&full[q], 4);
       mbar_init(&empty[q], 1);
     }
     mbar_init(&tfull[0], 1);
@@ -1374,14 +1443,11 @@ __global__ void __launch_bounds__(9 * kWarp)
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ producers --
-    const int t = threadIdx.x - 4 * kWarp;
-    const int kn = t >> 2, quarter = t & 3;         // neuron of the chunk, quarter of its 256-byte segment
+    // Warp 4 + p issues neurons 8p .. 8p + 7 of every stage; its lanes 0-7
+    // keep each its neuron's index four stages ahead (a ring of registers).
+    const int p = warp - 4;
+    const int kn = 8 * p + (lane & 7);
     const uint64_t pol = l2_evict_first();
-    // The neuron of each stage is loaded four stages ahead (a ring of four
-    // registers): a stage's copies need its index, and loading it when the
-    // stage is issued exposed one L2 round trip per stage.  pw / pqi walk this
-    // CTA's stages in issue order (items w = blockIdx.x + G i that have
-    // chunks, their chunks in order); -1: no neuron.
     int pw = blockIdx.x, pqi = 0, pq0 = 0, pnq = pw < items ? item_chunks(pw, pq0) : 0;
     while (pw < items && pnq == 0) {
       pw += gridDim.x;
@@ -1402,55 +1468,53 @@ __global__ void __launch_bounds__(9 * kWarp)
       return raw;
     };
     int kr0 = next_index(), kr1 = next_index(), kr2 = next_index(), kr3 = next_index();
+    const uint32_t tx = (uint32_t)(4 * 512 + (p == 0 ? NG * 1024 : 0));
     bool ok = true;
-    int it = 0;                                      // stages issued so far (all items)
+    int it = 0, issued = 0;
     for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
       const int col0 = (w % R) * kTcRows;
       int q0;
       const int nq = item_chunks(w, q0);
-      for (int qi = 0; qi < nq; ++qi, ++it) {
+      for (int qi = 0; qi < nq && ok; ++qi, ++it) {
         const int sl = it % NS;
-        if (it >= NS && !mbar_wait(&empty[sl], (uint32_t)((it / NS) - 1) & 1u, kWaitNs)) {
-          flag_error(err, kErrTimeout);
-          ok = false;
-          break;
-        }
-        unsigned char *st = stages + (size_t)sl * Ld::STAGE;
         const int q = q0 + qi;
         const int raw = kr0;
         kr0 = kr1;
         kr1 = kr2;
         kr2 = kr3;
         kr3 = next_index();
-        const int k = (unsigned)raw < (unsigned)n ? raw : -1;   // out of range: flagged by the gate/up kernel
-        const __half *rowp = WdT + (size_t)max(k, 0) * rs;
-        unsigned char *wt = st + (size_t)(kn >> 3) * 2048 + (size_t)(kn & 7) * 128;
+        const int k = (unsigned)raw < (unsigned)n ? raw : 0;   // padding / out of range: row 0, its a is zero
+        int rows[8];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int ci = quarter * 4 + cc;             // 16-byte chunk of the 256-byte segment
-          const int col = col0 + ci * 8;
-          const bool in = k >= 0 && col < d;
-          cp_async16(wt + (size_t)(ci >> 3) * 1024 + (((ci & 7) ^ (kn & 7)) << 4),
-                     in ? (const void *)(rowp + col) : (const void *)WdT, in ? 16u : 0u, pol);
+        for (int e = 0; e < 8; ++e) rows[e] = __shfl_sync(0xffffffffu, k, e);
+        if (lane == 0) {
+          if (it >= NS && !mbar_wait(&empty[sl], (uint32_t)((it / NS) - 1) & 1u, kWaitNs)) {
+            flag_error(err, kErrTimeout);
+            ok = false;
+          } else {
+            unsigned char *st = stages + (size_t)sl * Ld::STAGE;
+            mbar_arrive_expect_tx(&full[sl], tx);
+            // neurons 8p + 4h .. + 3: 8-neuron group p, rows 4h.. of its two 64-column atoms
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int atom = 0; atom < 2; ++atom)
+                tma_gather4(st + (size_t)p * 2048 + (size_t)atom * 1024 + (size_t)h * 512, &tm_w, col0 + atom * 64,
+                            rows[4 * h], rows[4 * h + 1], rows[4 * h + 2], rows[4 * h + 3], &full[sl], pol);
+            if (p == 0)
+#pragma unroll
+              for (int g = 0; g < NG; ++g)
+                tma_load_2d(st + Ld::W + (size_t)g * 1024, &tm_a, 0, (q * NG + g) * 16, &full[sl]);
+            issued = it + 1;
+          }
         }
-        unsigned char *at = st + Ld::W;
-        for (int qq = t; qq < NG * 16 * 4; qq += 4 * kWarp) {
-          const int row = qq >> 2, c = qq & 3;       // row 16 g + r of the NG group tiles
-          cp_async16(at + (size_t)(row >> 4) * 1024 + (row & 15) * 64 + ((c ^ (((row & 15) >> 1) & 3)) << 4),
-                     a2 + (((size_t)q * NG + (row >> 4)) * 16 + (row & 15)) * kTcChunk + c * 8, 16u);
-        }
-        cp_async_commit();
-        if (it >= NS - 1) {
-          cp_async_wait<NS - 1>();
-          fence_proxy_async_smem();
-          mbar_arrive(&full[(it - (NS - 1)) % NS]);
-        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
     }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (ok)
-      for (int e = max(0, it - (NS - 1)); e < it; ++e) mbar_arrive(&full[e % NS]);
+    // after a wait gave up, let each slot's last load land (bounded) before
+    // the shared memory is released
+    if (!ok && lane == 0)
+      for (int e = max(0, issued - NS); e < issued; ++e) mbar_wait(&full[e % NS], (uint32_t)(e / NS) & 1u, kWaitNs);
   } else if (warp == 8) {
     // ------------------------------------------------------------------ MMA --
     if (lane == 0) {
@@ -2678,12 +2742,58 @@ cudaError_t launch_final_reduce(const float *part, int G, int B, int d, float *y
 // CUDA-core pair measured about twice as fast there.
 bool tc_ok(const asf_ffn *f, int B) { return f->wdtype == ASF_F16 && B > 4 && B <= ASF_MAX_BATCH; }
 
+// cuTensorMapEncodeTiled, from the driver through the runtime (no link to the
+// driver library).
+using TmapEncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+TmapEncodeFn tmap_encoder() {
+  static TmapEncodeFn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (TmapEncodeFn) nullptr;
+    return reinterpret_cast<TmapEncodeFn>(p);
+  }();
+  return fn;
+}
+
+// Map of `rows` fp16 rows of d elements, `stride` elements apart, read in boxes
+// of box_cols columns x box_rows rows (box_cols * 2 bytes = the swizzle span:
+// the 128-byte swizzle for 64 columns, the 64-byte one for 32); out-of-range
+// rows and columns read as zeros, L2 filled from DRAM in 256-byte pieces.
+bool fp16_rows_map(CUtensorMap *tm, const void *base, int d, long long rows, long long stride, int box_rows,
+                   int box_cols = kTcK) {
+  TmapEncodeFn enc = tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)stride * sizeof(__half)};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool REGLU>
 cudaError_t launch_gu_tc(const asf_ffn *f, const __half *x, int Bh, int Btot, int g0, const int32_t *idx,
                          const int32_t *count, float *a, __half *a2, Header *hdr, cudaStream_t st) {
+  // TMA gathers for ReGLU rows longer than 8 KB (measured: +16-19% at d = 8192,
+  // 2-14% slower at d = 4096); the cp.async gathers otherwise
+  const int use_tma = REGLU && (size_t)f->d * sizeof(__half) > 8192;
+  CUtensorMap tmg, tmu, tmx;
+  std::memset(&tmg, 0, sizeof(tmg));
+  std::memset(&tmu, 0, sizeof(tmu));
+  std::memset(&tmx, 0, sizeof(tmx));
+  if (use_tma && (!fp16_rows_map(&tmg, f->Wg, f->d, f->n, ffn_rs(f), 1) ||
+                  !fp16_rows_map(&tmu, f->Wu, f->d, f->n, ffn_rs(f), 1) ||
+                  !fp16_rows_map(&tmx, x, f->d, Bh, f->d, kTcN)))
+    return cudaErrorInvalidValue;
   return launch(k_gu_tc<kTcN, REGLU>, dim3(std::min(sm_count(), kMaxGrid)), dim3(9 * kWarp),
-                GuTc<kTcN, REGLU>::SMEM, st, (const __half *)f->Wg, (const __half *)f->Wu, f->bias, x, f->d,
-                ffn_rs(f), f->n, Bh, idx, count, a, a2, Btot, g0, hdr);
+                GuTc<kTcN, REGLU>::SMEM, st, tmg, tmu, tmx, use_tma, (const __half *)f->Wg, (const __half *)f->Wu,
+                f->bias, x, f->d, ffn_rs(f), f->n, Bh, idx, count, a, a2, Btot, g0, hdr);
 }
 
 template <int NG>
@@ -2691,8 +2801,14 @@ cudaError_t launch_down_tc(const asf_ffn *f, int B, const int32_t *idx, const in
                            float *part, Header *hdr, cudaStream_t st) {
   const int R = tc_ranges(f), S = tc_splits(f);
   const int grid = std::min(std::min(sm_count(), kMaxGrid), R * S);
-  return launch(k_down_tc<NG>, dim3(grid), dim3(9 * kWarp), DnTc<NG>::SMEM, st, (const __half *)f->WdT, a2, idx,
-                count, f->d, ffn_rs(f), f->n, B, R, S, part, hdr);
+  // a2 as rows of 32 fp16 (64 bytes, 64-byte swizzle): chunk q, token group g at rows (q * NG + g) * 16
+  CUtensorMap tmw, tma;
+  const long long a2_rows = (long long)((f->n + kTcChunk - 1) / kTcChunk) * NG * 16;
+  if (!fp16_rows_map(&tmw, f->WdT, f->d, f->n, ffn_rs(f), 1) ||
+      !fp16_rows_map(&tma, a2, kTcChunk, a2_rows, kTcChunk, 16, kTcChunk))
+    return cudaErrorInvalidValue;
+  return launch(k_down_tc<NG>, dim3(grid), dim3(9 * kWarp), DnTc<NG>::SMEM, st, tmw, tma, idx, count, f->d, f->n, B,
+                R, S, part, hdr);
 }
 
 cudaError_t run_tc(const asf_ffn *f, const void *x, int B, const int32_t *idx, const int32_t *count, float *y,

@@ -215,6 +215,31 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------ tensor-map (TMA) loads --
+// A tensor map is a kernel parameter (const __grid_constant__ CUtensorMap);
+// these take its generic address.  No multicast.
+//
+// 2-D tile load of the box at (x, y) into shared memory, completing its bytes
+// on bar.  x * element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+// Four rows (y0..y3, any order) of a map whose box is one row high, columns
+// x.. of the box width, written as four consecutive box rows at dst (the
+// swizzle follows the shared-memory address).
+__device__ __forceinline__ void tma_gather4(void *dst, const void *tmap, int x, int y0, int y1, int y2, int y3,
+                                            uint64_t *bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
 // ----------------------------------------------------- tcgen05 (sm_100a) --
 // Tensor memory: allocated by one whole warp, address written to shared memory.
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {

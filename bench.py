@@ -556,7 +556,7 @@ def run_ours(args, cfg):
                                       f"timed alone with CUDA events around it in a captured graph",
             "achieved": ffn_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": ffn_gbs / hbm_peak,
             "peak_source": ("measured: MEASURED_PEAKS.json hbm_gbs (burst copy)" if peak_src == "measured" else
-                            "fallback: 6650 GB/s from the profiling recipe (MEASURED_PEAKS.json absent)"),
+                            "fallback: 6650 GB/s, an earlier STREAM-style copy measurement on B200 (MEASURED_PEAKS.json absent)"),
             "frac_of_nominal_7700": ffn_gbs / NOMINAL_HBM_GBS,
             "traffic": traffic_per_launch(tr, ffn_bytes_prof / (nprof * L)),
             "traffic_source": (tr or {}).get("source"),

@@ -52,7 +52,7 @@ def test_source_key_ignores_comments_but_not_code(bench, tmp_path):
 
 def test_traffic_record_is_used_only_for_the_kernels_it_measured(bench):
     rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
-    r = bench.traffic_record("llama2_7b_reglu:B1:predict")
+    r = bench.traffic_record("llama70b_reglu:B1:predict")
     if rec["source_sha"] == bench.source_sha():
         assert r is not None and 1.0 <= r["dram_bytes_per_algorithmic_byte"] < 1.01
     else:
